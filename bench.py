@@ -1,0 +1,625 @@
+#!/usr/bin/env python3
+"""Throughput of the W4A16 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl w4|reference] [--workload NAME]
+
+One step is one pass of the whole path over one batch of its workload: every
+weight matrix of the workload is quantized and packed (w4_quant_pack), and
+every activation batch is multiplied by its packed weight (w4a16_gemm).
+
+  decode (default)  M=1, K=4096, N in {4096, 11008, 12288}, asymmetric INT4 g=128:
+                    3 x (w4_quant_pack + w4a16_gemm); value = algorithmic GB/s
+  smallbatch        K=8192, N=28672, symmetric g=128: 1 x w4_quant_pack + M in {2,4,8,16,32}
+  prefill           K=4096, N=14336, asymmetric g=128: 1 x w4_quant_pack + M in {512,2048,8192};
+                    value = GEMM TFLOP/s over the step
+  quantizer         W[28672, 8192]: g in {32,64,128} x {sym, asym} + smoothing fold
+
+The K timed steps are captured in one CUDA graph and replayed once between
+CUDA events on the launching stream; event-record nodes between the kernels
+give each kernel's device time inside that same replay.  Inputs rotate over
+two sets so that no kernel finds its inputs in the 126 MB L2: each GEMM reads
+the weights packed one step earlier, after more than 126 MB of other traffic.
+
+Under torchrun (N > 1) every rank runs its own replica with its own seeds
+(weak scaling, no collective on the data path); the timed region is bracketed
+by barriers and the reported time is the max over ranks.  Rank 0 prints one
+JSON line.  ``--impl reference`` times the CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_gemm_quant_b200 import roofline, synth  # noqa: E402
+
+METRIC = "W4A16 g128 GEMV HBM GB/s (% peak); GEMM TFLOPS (% peak); quant-pack GB/s"
+KERNEL_SOURCES = {"w4_quant_pack": "quant_pack.cu", "w4a16_gemv": "gemv.cu", "w4a16_gemm_tc": "gemm_tc.cu"}
+THROTTLE_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["w4", "reference"], default="w4")
+    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer"], default="decode")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- ranks --
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def aggregate(local_ms: float, local_units: float, device=None):
+    """Max of the timed milliseconds and sum of the work units over all ranks."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return local_ms, local_units
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([float(local_units)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------ workloads --
+
+def problems_for(workload: str):
+    """Problems of a workload and how their weights are shared.
+
+    Returns a list of (weight_key, Problem); problems with the same key use one
+    quantization of one weight matrix per step."""
+    probs = synth.workload(workload)
+    if workload == "decode":
+        return [(p.name, p) for p in probs]
+    if workload in ("smallbatch", "prefill"):
+        return [("W", p) for p in probs]
+    return [(p.name, p) for p in probs]
+
+
+def kernel_name(M: int) -> str:
+    return "w4a16_gemv" if M <= 8 else "w4a16_gemm_tc"
+
+
+class Launch:
+    def __init__(self, name, work_bytes, flops, label):
+        self.name, self.bytes, self.flops, self.label = name, work_bytes, flops, label
+
+
+# ------------------------------------------------------------ cudart ----
+
+class CudaRT:
+    """The few runtime calls torch does not expose: external event-record
+    nodes inside a captured graph, and their elapsed times."""
+
+    def __init__(self):
+        self.L = ctypes.CDLL("libcudart.so.12")
+        self.L.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_uint]
+        self.L.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        self.L.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
+        self.L.cudaEventDestroy.argtypes = [ctypes.c_void_p]
+
+    def _check(self, rc, what):
+        if rc != 0:
+            raise RuntimeError("%s failed with cudaError %d" % (what, rc))
+
+    def event(self):
+        ev = ctypes.c_void_p()
+        self._check(self.L.cudaEventCreateWithFlags(ctypes.byref(ev), 0), "cudaEventCreateWithFlags")
+        return ev
+
+    def record_external(self, ev, stream_handle: int):
+        self._check(self.L.cudaEventRecordWithFlags(ev, ctypes.c_void_p(stream_handle), 1),
+                    "cudaEventRecordWithFlags")
+
+    def elapsed_ms(self, a, b) -> float:
+        ms = ctypes.c_float()
+        self._check(self.L.cudaEventElapsedTime(ctypes.byref(ms), a, b), "cudaEventElapsedTime")
+        return float(ms.value)
+
+    def destroy(self, ev):
+        self.L.cudaEventDestroy(ev)
+
+
+# ------------------------------------------------------------ clocks ----
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+        self.t_begin = self.t_end = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="w4clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def mark_begin(self):
+        self.t_begin = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvidia-smi unavailable"}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        win = [r for r in rows if self.t_begin is not None and self.t_begin - 1 <= r[0] <= self.t_end + 1] or rows
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in win for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in win), "sm_max_mhz": max(r[2] for r in win),
+                "reasons": reasons, "samples": len(win), "window": "sustained load before and during the timed replay"}
+
+
+def smi_gpu_id(local_rank: int) -> str:
+    """nvidia-smi index of this rank's device (honours CUDA_VISIBLE_DEVICES)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------ traffic ---
+
+def traffic_table() -> dict:
+    """DRAM bytes per launch from the committed ncu summary, keyed by
+    (kernel, problem); entries whose kernel source changed since are dropped."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    shas = {}
+    for k, src in KERNEL_SOURCES.items():
+        p = os.path.join(ROOT, "bit_gemm_quant_b200", "csrc", src)
+        if os.path.exists(p):
+            shas[k] = hashlib.sha256(open(p, "rb").read()).hexdigest()[:12]
+    for line in open(path):
+        parts = line.split()
+        if len(parts) != 4 or parts[0].startswith("#"):
+            continue
+        kern, label, sha, nbytes = parts
+        if shas.get(kern) == sha:
+            out[(kern, label)] = float(nbytes)
+    return out
+
+
+# ------------------------------------------------------------- our arm ---
+
+def run_w4(args, rank, world, local_rank):
+    import torch
+    import bit_gemm_quant_b200 as w4
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    w4.lib()
+    pk = roofline.peaks(ROOT)
+    plist = problems_for(args.workload)
+    R = 2  # rotating input sets
+    rank_seed = 1000 * rank
+
+    # ---- inputs (host bits, then device) ----
+    host_W, host_X, host_s = {}, {}, {}
+    for key, p in plist:
+        if key not in host_W:
+            host_W[key] = [synth.weights(p.seed + rank_seed + 17 * r, p.N, p.K, p.w_std, *p.w_outlier) for r in range(R)]
+            host_s[key] = p.s()
+        if p.M > 0:
+            host_X[p.name] = [synth.activations(p.seed + rank_seed + 17 * r, p.M, p.K, *p.x_outlier,
+                                                fixed_channels=p.x_fixed) for r in range(R)]
+    keys = list(dict.fromkeys(k for k, _ in plist))
+    first = {k: p for k, p in reversed(plist)}
+    qp = {k: first[k] for k in keys}     # the quantization problem of each weight key
+
+    def dev_bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16)
+
+    W_d = {k: [dev_bf16(b) for b in host_W[k]] for k in keys}
+    s_d = {k: (torch.from_numpy(host_s[k]).to(device) if host_s[k] is not None else None) for k in keys}
+    X_d = {n: [dev_bf16(b) for b in host_X[n]] for n in host_X}
+    packed = {}
+    for k in keys:
+        p = qp[k]
+        packed[k] = [w4.quant_pack(W_d[k][r], p.group, p.mode, s=s_d[k]) for r in range(R)]
+    Y_d, ws_d = {}, {}
+    for key, p in plist:
+        if p.M > 0:
+            Y_d[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device)
+            need = w4.w4a16_workspace_bytes(p.M, p.N, p.K, p.group)
+            ws_d[p.name] = torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
+    torch.cuda.synchronize()
+
+    launches = []
+    for k in keys:
+        p = qp[k]
+        launches.append(Launch("w4_quant_pack", roofline.quant_pack_bytes(p.N, p.K, p.group, p.mode, p.smooth), 0,
+                               k))
+        for key, pp in plist:
+            if key == k and pp.M > 0:
+                launches.append(Launch(kernel_name(pp.M), roofline.gemm_bytes(pp.M, pp.N, pp.K, pp.group, pp.mode),
+                                       roofline.gemm_flops(pp.M, pp.N, pp.K), pp.name))
+
+    def step(si, marks=None, rt=None, stream_handle=None):
+        r, r_prev = si % R, (si + 1) % R
+        i = 0
+        for k in keys:
+            p = qp[k]
+            if marks is not None:
+                rt.record_external(marks[i], stream_handle)
+            i += 1
+            w4.quant_pack(W_d[k][r], p.group, p.mode, s=s_d[k], out=packed[k][r])
+            for key, pp in plist:
+                if key == k and pp.M > 0:
+                    if marks is not None:
+                        rt.record_external(marks[i], stream_handle)
+                    i += 1
+                    q, sc, z = packed[k][r_prev]
+                    w4.gemm(X_d[pp.name][r], q, sc, z, pp.group, pp.mode, N=pp.N, workspace=ws_d[pp.name],
+                            out=Y_d[pp.name])
+
+    per_step = len(launches)
+    # ---- eager warm-up ----
+    for si in range(max(3, args.warmup)):
+        step(si)
+    torch.cuda.synchronize()
+
+    # ---- capture the K timed steps with event nodes between kernels ----
+    rt = CudaRT()
+    K = args.steps
+    marks = [rt.event() for _ in range(K * per_step + 1)]
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream(device)
+    cap_stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cap_stream):
+        h = torch.cuda.current_stream().cuda_stream
+        for si in range(K):
+            step(si, marks[si * per_step:(si + 1) * per_step], rt, h)
+        rt.record_external(marks[-1], h)
+    torch.cuda.synchronize()
+
+    # ---- sustained load (untimed) so the clock samples cover a steady state ----
+    sampler = ClockSampler(smi_gpu_id(local_rank))
+    sampler.start()
+    sampler.mark_begin()
+    t_end = time.time() + 1.5
+    replays = 0
+    while time.time() < t_end or replays < 2:
+        graph.replay()
+        replays += 1
+        torch.cuda.synchronize()
+
+    def timed():
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        e1.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
+
+    local_ms = timed()
+    sampler.mark_end()
+    clocks = sampler.stop()
+    if any(r in clocks.get("reasons", []) for r in THROTTLE_REASONS):
+        sampler = ClockSampler(sampler.gpu_id)
+        sampler.start()
+        sampler.mark_begin()
+        local_ms = timed()
+        sampler.mark_end()
+        clocks = sampler.stop()
+        clocks["remeasured"] = True
+
+    # per-kernel device time inside this replay
+    kt = {}
+    for si in range(K):
+        for j, L in enumerate(launches):
+            a = marks[si * per_step + j]
+            b = marks[si * per_step + j + 1]
+            kt.setdefault((L.name, L.label), []).append(rt.elapsed_ms(a, b))
+
+    step_bytes = sum(L.bytes for L in launches)
+    step_flops = sum(L.flops for L in launches)
+    work = K * (step_flops if args.workload == "prefill" else step_bytes)
+    max_ms, total_work = aggregate(local_ms, work, device)
+
+    if args.workload == "prefill":
+        value, unit = total_work / (max_ms * 1e-3) / 1e12, "TFLOP/s"
+    else:
+        value, unit = total_work / (max_ms * 1e-3) / 1e9, "GB/s"
+
+    # ---- per-kernel roofline ----
+    traffic = traffic_table()
+    timed_s = local_ms * 1e-3
+    kernels = {}
+    by_name = {}
+    for L in launches:
+        ts = kt[(L.name, L.label)]
+        avg = statistics.mean(ts)
+        ent = {"launches": len(ts), "avg_us": round(avg * 1e3, 3), "bytes": L.bytes,
+               "gbs": round(L.bytes / (avg * 1e-3) / 1e9, 1),
+               "hbm_frac": round(L.bytes / (avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        if L.flops:
+            tf = L.flops / (avg * 1e-3) / 1e12
+            peak_t = pk["bf16_tflops_sustained"] if timed_s >= 1.0 else pk["bf16_tflops"]
+            ent.update({"flops": L.flops, "tflops": round(tf, 1), "tensor_frac": round(tf / peak_t, 4)})
+        kernels["%s[%s]" % (L.name, L.label)] = ent
+        by_name.setdefault(L.name, []).append((L, ts))
+
+    dom = max(by_name, key=lambda n: sum(sum(ts) for _, ts in by_name[n]))
+    dom_launches = by_name[dom]
+    tot_time = sum(sum(ts) for _, ts in dom_launches) * 1e-3
+    nlaunch = sum(len(ts) for _, ts in dom_launches)
+    if dom == "w4a16_gemm_tc":
+        per_launch = sum(L.flops * len(ts) for L, ts in dom_launches) / nlaunch
+        peak = pk["bf16_tflops_sustained"] if timed_s >= 1.0 else pk["bf16_tflops"]
+        achieved = per_launch / (tot_time / nlaunch) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4)}
+    else:
+        per_launch = sum(L.bytes * len(ts) for L, ts in dom_launches) / nlaunch
+        achieved = per_launch / (tot_time / nlaunch) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4)}
+    tr = [traffic.get((dom, L.label)) for L, _ in dom_launches]
+    roof["traffic"] = (sum(tr) / len(tr)) if tr and all(t is not None for t in tr) else None
+    roof["kernel"] = dom
+    roof["peak_source"] = "%s (%s)" % (pk["source"], "MEASURED_PEAKS.json" if pk["source"] == "measured" else "recipe")
+    roof["algorithmic_per_launch"] = per_launch
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, min(args.steps, 10))
+        e2e_ms, e2e_work = aggregate(e2e["ms"], e2e["work"] if args.workload != "prefill" else e2e["flops"], device)
+        e2e = {"value": round(e2e_work / (e2e_ms * 1e-3) / (1e12 if args.workload == "prefill" else 1e9), 2),
+               "unit": unit, "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+               "steps": e2e["steps"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload, plist, keys, qp, host_W, host_X, host_s, args.cpu_budget)
+
+    for ev in marks:
+        rt.destroy(ev)
+    del graph
+    if rank == 0:
+        wl_desc = {
+            "decode": "decode GEMV: M=1, K=4096, N in {4096,11008,12288}, asymmetric INT4 g=128, fp16 scales, uint4 zero-points; step = w4_quant_pack + w4a16_gemm per layer",
+            "smallbatch": "small-batch decode: K=8192, N=28672, symmetric INT4 g=128, M in {2,4,8,16,32}; step = 1 w4_quant_pack + 5 w4a16_gemm",
+            "prefill": "prefill GEMM: K=4096, N=14336, asymmetric INT4 g=128, M in {512,2048,8192}; step = 1 w4_quant_pack + 3 w4a16_gemm",
+            "quantizer": "quantizer sweep: W[28672,8192], g in {32,64,128} x {sym,asym} + smoothing fold; step = 7 w4_quant_pack",
+        }[args.workload]
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K,
+            "warmup": max(3, args.warmup) + replays, "ms_per_step": round(max_ms / K, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl_desc, "codes": "int4 packed 8 per uint32", "accumulate": "fp32",
+                       "l2": "inputs rotate over 2 sets; each kernel's inputs were last touched before >126 MB of other traffic",
+                       "timing": "K steps captured in one CUDA graph, replayed between CUDA events on the launching stream; max over ranks",
+                       "parallelism": "replicas (dp%d), no data-path collective" % world},
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": K * per_step * world, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps):
+    """Same step through the tensor API with pinned host inputs and outputs:
+    host->device copies of each step's weights and activations, the library
+    calls, and device->host copies of the packed weights and Y, all timed."""
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).pin_memory()
+    hW = {k: pin(host_W[k][0]) for k in keys}
+    hX = {n: pin(v[0]) for n, v in host_X.items()}
+    hs = {k: (torch.from_numpy(host_s[k]).pin_memory() if host_s[k] is not None else None) for k in keys}
+    outs = {}
+    h2d = sum(hW[k].numel() * 2 + (hs[k].numel() * 4 if hs[k] is not None else 0) for k in keys) + \
+        sum(x.numel() * 2 for x in hX.values())
+    d2h = 0
+    for k in keys:
+        p = qp[k]
+        qs, ss, zs = w4.packed_shapes(p.N, p.K, p.group)
+        outs[k] = (torch.empty(qs, dtype=torch.int32).pin_memory(), torch.empty(ss, dtype=torch.float16).pin_memory(),
+                   torch.empty(zs, dtype=torch.int32).pin_memory() if p.mode == 1 else None)
+        d2h += sum(t.numel() * t.element_size() for t in outs[k] if t is not None)
+    for key, p in plist:
+        if p.M > 0:
+            outs[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
+            d2h += p.M * p.N * 2
+    work = sum(roofline.quant_pack_bytes(qp[k].N, qp[k].K, qp[k].group, qp[k].mode, qp[k].smooth) for k in keys) + \
+        sum(roofline.gemm_bytes(p.M, p.N, p.K, p.group, p.mode) for _, p in plist if p.M > 0)
+    flops = sum(roofline.gemm_flops(p.M, p.N, p.K) for _, p in plist if p.M > 0)
+
+    def one():
+        for k in keys:
+            p = qp[k]
+            Wd = hW[k].to(device, non_blocking=True).view(torch.bfloat16)
+            sd = hs[k].to(device, non_blocking=True) if hs[k] is not None else None
+            q, sc, z = w4.quant_pack(Wd, p.group, p.mode, s=sd)
+            for t_h, t_d in zip(outs[k], (q, sc, z)):
+                if t_h is not None:
+                    t_h.copy_(t_d, non_blocking=True)
+            for key, pp in plist:
+                if key == k and pp.M > 0:
+                    Xd = hX[pp.name].to(device, non_blocking=True).view(torch.bfloat16)
+                    Y = w4.gemm(Xd, q, sc, z, pp.group, pp.mode, N=pp.N)
+                    outs[pp.name].copy_(Y, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    e1.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    return {"ms": ms, "work": work * steps, "flops": flops * steps, "h2d": h2d, "d2h": d2h, "steps": steps}
+
+
+# ------------------------------------------------------- oracle (CPU) ---
+
+def oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_per_weight: int, offset: int = 0):
+    """Run the oracle on rows [offset, offset + r) of each weight of the
+    workload: quantize and pack, dequantize, and the fp64 product for those
+    output channels.  Returns the algorithmic bytes (or flops) processed."""
+    nbytes = 0
+    nflops = 0
+    for k in keys:
+        p = qp[k]
+        W = host_W[k][0]
+        r0 = offset % p.N
+        r1 = min(p.N, r0 + rows_per_weight)
+        q, sc, z = oracle.quant_pack(W, p.group, p.mode, s=host_s[k], rows=(r0, r1))
+        nbytes += roofline.quant_pack_bytes(r1 - r0, p.K, p.group, p.mode, p.smooth)
+        users = [pp for key, pp in plist if key == k and pp.M > 0]
+        if users:
+            what = oracle.dequant(q, sc, z, p.K, p.group, p.mode, rows=(r0, r1))
+            for pp in users:
+                oracle.gemm_f64(host_X[pp.name][0], what)
+                nbytes += roofline.gemm_bytes(pp.M, r1 - r0, pp.K, pp.group, pp.mode)
+                nflops += roofline.gemm_flops(pp.M, r1 - r0, pp.K)
+    return nbytes, nflops
+
+
+def cpu_baseline(workload, plist, keys, qp, host_W, host_X, host_s, budget_s):
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, 4)
+    dt = time.perf_counter() - t0
+    rows = max(4, int(4 * budget_s / max(dt, 1e-3)))
+    rows = min(rows, max(p.N for p in qp.values()))
+    t0 = time.perf_counter()
+    nbytes, nflops = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows)
+    dt = time.perf_counter() - t0
+    if workload == "prefill":
+        val, unit = nflops / dt / 1e12, "TFLOP/s"
+    else:
+        val, unit = nbytes / dt / 1e9, "GB/s"
+    return {"value": val, "unit": unit, "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
+            "sample": "first %d rows of each weight of the workload: oracle fold+quantize+pack, dequantize and "
+                      "fp64 product for those output channels, single thread" % rows}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    plist = problems_for(args.workload)
+    keys = list(dict.fromkeys(k for k, _ in plist))
+    first = {k: p for k, p in reversed(plist)}
+    qp = {k: first[k] for k in keys}
+    host_W = {k: [synth.weights(qp[k].seed, qp[k].N, qp[k].K, qp[k].w_std, *qp[k].w_outlier)] for k in keys}
+    host_s = {k: qp[k].s() for k in keys}
+    host_X = {p.name: [p.X()] for _, p in plist if p.M > 0}
+    rows = 8
+    for si in range(max(3, args.warmup)):
+        oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, si * rows)
+    nb = nf = 0
+    t0 = time.perf_counter()
+    for si in range(args.steps):
+        b, f = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, si * rows)
+        nb, nf = nb + b, nf + f
+    dt = time.perf_counter() - t0
+    if args.workload == "prefill":
+        val, unit = nf / dt / 1e12, "TFLOP/s"
+    else:
+        val, unit = nb / dt / 1e9, "GB/s"
+    sample = ("%d rows of each weight per step (rotating): oracle fold+quantize+pack, dequantize and fp64 "
+              "product for those output channels, single thread" % rows)
+    out = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
+           "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": dt * 1e3 / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
+           "data": "synthetic", "config": {"workload": args.workload, "kind": "CPU oracle on a bounded sample"},
+           "cpu_baseline": {"value": val, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+           "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return 0
+    run_w4(args, rank, world, local_rank)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

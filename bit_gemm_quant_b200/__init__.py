@@ -1,1 +1,135 @@
-"""B200-native group-wise INT4 weight quantization and W4A16 GEMV/GEMM."""
+"""B200-native group-wise INT4 weight quantization and the W4A16 GEMV/GEMM.
+
+A thin ctypes binding over the C ABI of ``libw4.so`` (declared in
+``include/w4.h``).  The raw entry points keep their C names and take device
+pointers as integers; the tensor helpers ``quant_pack`` and ``gemm`` only
+allocate outputs with torch, pass ``data_ptr()`` values and the current CUDA
+stream, and raise ``W4Error`` on a nonzero status.  Every step of the path
+runs in the library's kernels; there is no fallback: if ``libw4.so`` is
+missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+SYM, ASYM = 0, 1
+W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
+_lib = None
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s failed: %s" % (what, w4_status_string(status) if _lib else status))
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libw4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError("libw4.so is not built; run `python -m bit_gemm_quant_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.w4_quant_pack.argtypes = [P, I64, I64, I, I, P, P, P, P, P]
+        L.w4_quant_pack.restype = I
+        L.w4a16_workspace_bytes.argtypes = [I64, I64, I64, I]
+        L.w4a16_workspace_bytes.restype = SZ
+        L.w4a16_gemm.argtypes = [P, I64, I64, I64, P, P, P, I, I, P, P, SZ, P]
+        L.w4a16_gemm.restype = I
+        L.w4_status_string.argtypes = [I]
+        L.w4_status_string.restype = ctypes.c_char_p
+        L.w4_layout_version.argtypes = []
+        L.w4_layout_version.restype = I
+        L.w4_device_error.argtypes = [ctypes.POINTER(I)]
+        L.w4_device_error.restype = I
+        _lib = L
+    return _lib
+
+
+# --- raw C ABI, same names and argument order as include/w4.h ----------------
+
+def w4_quant_pack(W, N, K, group, mode, s, qweight, scales, qzeros, stream) -> int:
+    return lib().w4_quant_pack(W, N, K, group, mode, s, qweight, scales, qzeros, stream)
+
+
+def w4a16_workspace_bytes(M, N, K, group) -> int:
+    return int(lib().w4a16_workspace_bytes(M, N, K, group))
+
+
+def w4a16_gemm(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace, workspace_bytes, stream) -> int:
+    return lib().w4a16_gemm(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace,
+                            workspace_bytes, stream)
+
+
+def w4_status_string(status: int) -> str:
+    return lib().w4_status_string(int(status)).decode()
+
+
+def w4_layout_version() -> int:
+    return int(lib().w4_layout_version())
+
+
+def w4_device_error() -> int:
+    code = ctypes.c_int(0)
+    st = lib().w4_device_error(ctypes.byref(code))
+    if st != W4_OK:
+        raise W4Error(st, "w4_device_error")
+    return code.value
+
+
+# --- torch tensor helpers (argument marshalling only) -------------------------
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def packed_shapes(N: int, K: int, group: int):
+    G = K // group
+    return (N, K // 8), (N, G), (N, (G + 7) // 8)
+
+
+def quant_pack(W, group: int = 128, mode: int = SYM, s=None, stream=None, out=None):
+    """Quantize a bf16 CUDA tensor W[N,K]; returns (qweight, scales, qzeros or None)."""
+    import torch
+    N, K = W.shape
+    qs, ss, zs = packed_shapes(N, K, group)
+    if out is None:
+        qweight = torch.empty(qs, dtype=torch.int32, device=W.device)
+        scales = torch.empty(ss, dtype=torch.float16, device=W.device)
+        qzeros = torch.empty(zs, dtype=torch.int32, device=W.device) if mode == ASYM else None
+    else:
+        qweight, scales, qzeros = out
+    st = w4_quant_pack(_ptr(W), N, K, group, mode, _ptr(s), _ptr(qweight), _ptr(scales), _ptr(qzeros),
+                       _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_quant_pack")
+    return qweight, scales, qzeros
+
+
+def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None, workspace=None,
+         out=None, stream=None):
+    """Y[M,N] = X . W^T from the packed weight; X bf16 CUDA tensor [M,K]."""
+    import torch
+    M, K = X.shape
+    if N is None:
+        N = qweight.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = w4a16_workspace_bytes(M, N, K, group)
+    if need and workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=X.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = w4a16_gemm(_ptr(X), M, N, K, _ptr(qweight), _ptr(scales), _ptr(qzeros), group, mode, _ptr(Y),
+                    _ptr(workspace), wbytes, _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4a16_gemm")
+    return Y

@@ -1,0 +1,87 @@
+// extern "C" entry points of libw4 (declared in include/w4.h): argument
+// validation on the host, then dispatch to the kernels.  Nothing here
+// allocates device memory or synchronizes a stream.
+#include "common.cuh"
+
+namespace {
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
+
+bool mode_ok(int m) { return m == W4_SYM || m == W4_ASYM; }
+
+// int64 products used for sizes must not overflow
+bool fits(int64_t a, int64_t b) { return a > 0 && b > 0 && a <= INT64_MAX / b; }
+
+}  // namespace
+
+extern "C" {
+
+const char *w4_status_string(int status)
+{
+    switch (status) {
+    case W4_OK: return "W4_OK";
+    case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG: null or misaligned pointer, bad size, group or mode";
+    case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED: well-formed request outside what the kernels cover";
+    case W4_ERR_CUDA: return "W4_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    default: return "unknown w4 status";
+    }
+}
+
+int w4_layout_version(void) { return W4_LAYOUT_VERSION; }
+
+w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode, const float *s,
+                        uint32_t *qweight, void *scales, uint32_t *qzeros, w4_stream_t stream)
+{
+    if (!W || !qweight || !scales) return W4_ERR_INVALID_ARG;
+    if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
+    if (N < 1 || K < 8 || K % group != 0 || !fits(N, K)) return W4_ERR_INVALID_ARG;
+    if ((mode == W4_ASYM) != (qzeros != nullptr)) return W4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 2)) return W4_ERR_INVALID_ARG;
+    if (s && !aligned(s, 16)) return W4_ERR_INVALID_ARG;
+    if (qzeros && !aligned(qzeros, 4)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e =
+        w4::launch_quant_pack(W, N, K, group, mode, s, qweight, scales, qzeros, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group)
+{
+    (void)M; (void)N; (void)K; (void)group;
+    return 0;
+}
+
+w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                     const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
+                     void *workspace, size_t workspace_bytes, w4_stream_t stream)
+{
+    if (!X || !qweight || !scales || !Y) return W4_ERR_INVALID_ARG;
+    if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N))
+        return W4_ERR_INVALID_ARG;
+    if ((mode == W4_ASYM) != (qzeros != nullptr)) return W4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(Y, 2))
+        return W4_ERR_INVALID_ARG;
+    if (qzeros && !aligned(qzeros, 4)) return W4_ERR_INVALID_ARG;
+    const size_t need = w4a16_workspace_bytes(M, N, K, group);
+    if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256))))
+        return W4_ERR_INVALID_ARG;
+    if (N > (int64_t)INT32_MAX * 16) return W4_ERR_UNSUPPORTED;
+    cudaError_t e;
+    if (M <= 8) {
+        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, Y, (cudaStream_t)stream);
+    } else {
+        return W4_ERR_UNSUPPORTED;
+    }
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_device_error(int *code)
+{
+    if (!code) return W4_ERR_INVALID_ARG;
+    *code = 0;
+    return W4_OK;
+}
+
+}  // extern "C"

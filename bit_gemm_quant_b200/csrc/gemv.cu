@@ -1,0 +1,219 @@
+// w4a16_gemm, M <= 8: the decode GEMV / skinny path.
+//
+// Method: page 2 (learn.longtimenohack.com .../quantization.html) opens with
+// "reading weights is the top cost of decode", page 4
+// (llm-glossary.tokens-kit.com/terms/quantization-methods/, GPTQ section) with
+// "small-batch decode profits from the weight bandwidth", and page 3
+// (blog.freezetheflame.cc quantization deep dive) section 1.2 with "fuse
+// dequantize into the GEMM so the weights stay 4-bit in HBM"; section 3.1 of
+// the same page sketches Marlin, which unpacks INT4 in registers and feeds
+// mma.sync.  Dequantization follows page 5 (ai-infra.cypggs.com
+// .../02-core-ideas) section 2.2, x^ = (q - zp) * s, rounded once to bf16.
+//
+// Design (HBM-bound: 0.5 B of codes + 1/64 B of scale per weight at g = 128):
+//   * a CTA owns 16 output channels and all of K; its 8 warps split K into
+//     512-wide super-chunks (warp w takes super-chunks w, w+8, ...), and sum
+//     their partial tiles in shared memory at the end (no global scratch);
+//   * lane (g, t) = (lane/4, lane%4) of a warp loads, for channels g and g+8,
+//     the 64 contiguous bytes (128 codes) at k = 512*sc + 128*t: all of its
+//     loads are issued before any arithmetic (8 x 16 B per lane);
+//   * each 32-bit word of codes gives four bf16x2 pairs of ADJACENT elements
+//     with one shift and one LOP3 (the packed layout keeps even elements in
+//     the low half-word), as 128 + u via the bf16 exponent of 128;
+//   * exact w^ = bf16_rne((u - zp) * s16) with three bf16x2 operations:
+//     D = (128+u) - (128+zp) (exact), c = D * s_lo (exact: <= 7 bits) and
+//     w^ = fma(D, s_hi, c), where s16 = s_hi + s_lo splits the fp16 scale into
+//     its bf16 rounding and the (<= 3-bit) remainder; the fused multiply-add
+//     rounds the exact product D * s16 once;
+//   * mma.sync m16n8k16 (bf16 in, fp32 accumulate) takes those registers as
+//     its A fragment directly: the k-order inside an MMA is free, so a
+//     thread's logical columns (2t, 2t+1) and (2t+8, 2t+9) are mapped to the
+//     physical elements 8w+4h+{0,1} and 8w+4h+{2,3} of its own words, and the
+//     activation fragment for token g is then the plain 16-byte chunk
+//     X[g][k + 8w .. k + 8w + 7];
+//   * tokens occupy the MMA's N = 8 columns; lanes with g >= M feed zeros.
+#include "common.cuh"
+
+namespace w4 {
+namespace {
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Per-(channel, group) dequantization constants, each duplicated into both
+// halves of a bf16x2: s_hi = bf16_rne(s16), s_lo = s16 - s_hi, Z = 128 + zp.
+struct GroupConst {
+    uint32_t shi, slo, z;
+};
+
+__device__ __forceinline__ GroupConst group_const(unsigned short s16bits, int zp)
+{
+    const float sf = __half2float(__ushort_as_half(s16bits));
+    const __nv_bfloat16 hi = __float2bfloat16_rn(sf);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(sf - __bfloat162float(hi));   // exact
+    const uint32_t h = __bfloat16_as_ushort(hi), l = __bfloat16_as_ushort(lo);
+    GroupConst gc;
+    gc.shi = h | (h << 16);
+    gc.slo = l | (l << 16);
+    gc.z = 0x43004300u | ((uint32_t)zp << 16) | (uint32_t)zp;
+    return gc;
+}
+
+// w^ for elements (8c+2j, 8c+2j+1) of packed word q.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupConst &gc)
+{
+    const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) | 0x43004300u;   // 128 + u, as bf16x2
+    const uint32_t D = bf2_sub(v, gc.z);
+    return bf2_fma(D, gc.shi, bf2_mul(D, gc.slo));
+}
+
+constexpr int kWarps = 8;
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(kWarps * 32)
+gemv_kernel(const uint4 *__restrict__ X, int M, int64_t N, int64_t K, const uint4 *__restrict__ qweight,
+            const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
+            __nv_bfloat16 *__restrict__ Y)
+{
+    constexpr int QPG = G / 32;                  // 32-code chunks per group
+    __shared__ float red[kWarps][32][4];
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t rowA = (int64_t)blockIdx.x * 16 + g, rowB = rowA + 8;
+    const bool okA = rowA < N, okB = rowB < N;
+    const int64_t KQ = K >> 5;                   // 16-byte code chunks per channel
+    const int64_t NG = K / G, ZW = (NG + 7) >> 3;
+    const bool has_x = g < M;
+    const uint4 *xrow = X + (int64_t)(has_x ? g : 0) * (K >> 3);
+
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+
+    for (int64_t sc = warp; sc * 16 < KQ; sc += kWarps) {
+        const int64_t q0 = sc * 16 + t * 4;      // first chunk of this lane
+        uint4 qa[4], qb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const bool ok = q0 + i < KQ;
+            qa[i] = (ok && okA) ? ld_stream(qweight + rowA * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+            qb[i] = (ok && okB) ? ld_stream(qweight + rowB * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        GroupConst ca, cb;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int64_t qi = q0 + i;
+            const bool ok = qi < KQ;
+            const int64_t k = qi * 32;
+            if (i % QPG == 0) {
+                const int64_t j = ok ? k / G : 0;
+                int za = 8, zb = 8;
+                if (MODE == W4_ASYM) {
+                    za = okA ? (int)((__ldg(qzeros + rowA * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu) : 0;
+                    zb = okB ? (int)((__ldg(qzeros + rowB * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu) : 0;
+                }
+                ca = group_const(okA ? __ldg(scales + rowA * NG + j) : (unsigned short)0, za);
+                cb = group_const(okB ? __ldg(scales + rowB * NG + j) : (unsigned short)0, zb);
+            }
+            uint4 xv[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                xv[w] = (has_x && ok) ? __ldg(xrow + (k >> 3) + w) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t wa[4] = {qa[i].x, qa[i].y, qa[i].z, qa[i].w};
+            const uint32_t wb[4] = {qb[i].x, qb[i].y, qb[i].z, qb[i].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t a0 = dequant_pair(wa[w], 0, ca), a1 = dequant_pair(wa[w], 1, ca);
+                const uint32_t a2 = dequant_pair(wa[w], 2, ca), a3 = dequant_pair(wa[w], 3, ca);
+                const uint32_t b0 = dequant_pair(wb[w], 0, cb), b1 = dequant_pair(wb[w], 1, cb);
+                const uint32_t b2 = dequant_pair(wb[w], 2, cb), b3 = dequant_pair(wb[w], 3, cb);
+                mma_bf16_16816(acc, a0, b0, a1, b1, xv[w].x, xv[w].y);
+                mma_bf16_16816(acc, a2, b2, a3, b3, xv[w].z, xv[w].w);
+            }
+        }
+    }
+
+    red[warp][lane][0] = acc[0];
+    red[warp][lane][1] = acc[1];
+    red[warp][lane][2] = acc[2];
+    red[warp][lane][3] = acc[3];
+    __syncthreads();
+    if (warp == 0) {
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[i] += red[w][lane][i];
+        const int m0 = 2 * t, m1 = 2 * t + 1;    // tokens of c0/c2 and c1/c3
+        if (okA && m0 < M) Y[(int64_t)m0 * N + rowA] = __float2bfloat16_rn(s[0]);
+        if (okA && m1 < M) Y[(int64_t)m1 * N + rowA] = __float2bfloat16_rn(s[1]);
+        if (okB && m0 < M) Y[(int64_t)m0 * N + rowB] = __float2bfloat16_rn(s[2]);
+        if (okB && m1 < M) Y[(int64_t)m1 * N + rowB] = __float2bfloat16_rn(s[3]);
+    }
+}
+
+template <int G, int MODE>
+cudaError_t launch_g_mode(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                          const void *scales, const uint32_t *qzeros, void *Y, cudaStream_t stream)
+{
+    const int64_t blocks = (N + 15) / 16;
+    gemv_kernel<G, MODE><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+        (const uint4 *)X, (int)M, N, K, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
+        (__nv_bfloat16 *)Y);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                        const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
+                        cudaStream_t stream)
+{
+    switch (group * 2 + mode) {
+    case 32 * 2 + W4_SYM: return launch_g_mode<32, W4_SYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
+    case 32 * 2 + W4_ASYM: return launch_g_mode<32, W4_ASYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
+    case 64 * 2 + W4_SYM: return launch_g_mode<64, W4_SYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
+    case 64 * 2 + W4_ASYM: return launch_g_mode<64, W4_ASYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
+    case 128 * 2 + W4_SYM: return launch_g_mode<128, W4_SYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
+    case 128 * 2 + W4_ASYM: return launch_g_mode<128, W4_ASYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace w4

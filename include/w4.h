@@ -1,0 +1,147 @@
+/*
+ * w4.h -- C ABI of libw4: group-wise INT4 weight quantization and the W4A16
+ * product on NVIDIA B200 (sm_100a).
+ *
+ * The method (web pages on LLM quantization, "page N" below):
+ *   page 5, ai-infra.cypggs.com .../model-quantization/02-core-ideas, section 2.2:
+ *     symmetric  q = clip(round(x/s), -8, 7),       s = max|x| / 7
+ *     asymmetric q = clip(round(x/s) + zp, 0, 15),  s = (max - min) / 15,
+ *                zp = round(-min/s)
+ *     dequantize x^ = (q - zp) * s, rounding is round-to-nearest-even.
+ *   page 2, learn.longtimenohack.com .../quantization.html, item (1) group
+ *     quantization: rows are cut into groups of g weights that share one fp16
+ *     scale and an integer zero-point (g = 128 gives 4.125 bits per weight).
+ *   page 3, blog.freezetheflame.cc .../quantization-deep-dive.html, section 1.2
+ *     (dequantize fused into the GEMM so weights stay 4-bit in memory), 2.2
+ *     (per-group scales have shape [C_out, num_groups]), 5.3 (the smoothing
+ *     vector s is folded into the weights offline, W * s, and the activations
+ *     are divided by s upstream).
+ *   page 5 section 2.4 and page 1 (AWQ): X' = X/s, W' = W * diag(s) leaves
+ *     X W^T unchanged.
+ *
+ * Exact semantics (fixed where the pages leave a step open):
+ *   w'   = fl32(float(w[n][k]) * s[k])        (w' = float(w) when s == NULL)
+ *   sym  : amax = max|w'| over the group, s32 = fl32(amax / 7)
+ *   asym : mn = min(0, min w'), mx = max(0, max w'), s32 = fl32(fl32(mx - mn) / 15)
+ *   s16  = fp16_rne(s32), saturated to 65504 (the stored scale)
+ *   zp   = sym: 8;  asym: clip(rint(fl32(-mn / s16)), 0, 15)   (0 when s16 == 0)
+ *   u    = sym: clip(rint(fl32(w' / s16)), -8, 7) + 8
+ *          asym: clip(rint(fl32(w' / s16)) + zp, 0, 15)
+ *          (the zero code, 8 or 0, when s16 == 0); rint = round half to even
+ *   w^   = bf16_rne(float(u - zp) * float(s16))   (the product is exact in fp32)
+ *   Y[m][n] = bf16_rne(sum_k x[m][k] * w^[n][k]) with fp32 accumulation.
+ *
+ * Packed layout, version W4_LAYOUT_VERSION (all arrays row-major, C order):
+ *   qweight  uint32 [N][K/8]:   word c of row n holds elements k = 8c..8c+7;
+ *            bits [4i, 4i+4) hold u of element 8c+2i and bits [16+4i, 16+4i+4)
+ *            hold u of element 8c+2i+1 (i = 0..3): even elements in the low
+ *            half-word, odd elements in the high half-word.
+ *   scales   fp16 [N][K/g]:     s16 of group j = k/g.
+ *   qzeros   uint32 [N][ceil(K/g/8)], asymmetric mode only: bits [4(j%8), 4(j%8)+4)
+ *            of word j/8 hold zp of group j; unused nibbles are 0.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned unless stated otherwise; the library allocates no device memory
+ *     and keeps no state between calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream).  Calls are asynchronous: the library never synchronizes.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and returns W4_ERR_INVALID_ARG or
+ *     W4_ERR_UNSUPPORTED.  A launch failure returns W4_ERR_CUDA.  No exception
+ *     crosses the ABI and the library never aborts the process.
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified codes.
+ *   - There is no CPU fallback: a shape the kernels do not cover is rejected.
+ */
+#ifndef W4_H
+#define W4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4_LAYOUT_VERSION 1
+
+/* A cudaStream_t (the runtime's stream handle type); NULL = default stream. */
+typedef struct CUstream_st *w4_stream_t;
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad group or mode   */
+    W4_ERR_UNSUPPORTED = 2,   /* well-formed request outside what the kernels cover     */
+    W4_ERR_CUDA = 3           /* a CUDA runtime call or launch failed                   */
+} w4_status;
+
+typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
+
+/*
+ * w4_quant_pack -- fold, group-quantize and pack a bf16 weight matrix.
+ *   (page 5 section 2.2 formulas; page 2 group quantization; page 3 sections
+ *    2.2 and 5.3 for the scale shape and the fold)
+ *   W        bf16 [N][K], row k-contiguous.
+ *   N, K     N >= 1; K >= 8, K % group == 0.
+ *   group    32, 64 or 128.
+ *   mode     W4_SYM or W4_ASYM.
+ *   s        fp32 [K] smoothing vector folded into W (w' = w * s[k]), or NULL.
+ *   qweight  out, uint32 [N][K/8] (layout above).
+ *   scales   out, fp16 [N][K/group]; only 2-byte alignment required.
+ *   qzeros   out, uint32 [N][ceil(K/group/8)]; must be NULL in W4_SYM mode and
+ *            non-NULL in W4_ASYM mode; only 4-byte alignment required.
+ * Every output byte is written; outputs must not overlap inputs.
+ */
+w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode, const float *s,
+                        uint32_t *qweight, void *scales, uint32_t *qzeros, w4_stream_t stream);
+
+/*
+ * w4a16_workspace_bytes -- device scratch that w4a16_gemm needs for this
+ * shape (split-K partial sums and tile counters), 0 if none.  The workspace
+ * must be zero-filled before its first use with a given shape; every
+ * successful call leaves it zero-filled again, so one zeroed buffer can be
+ * reused across calls on the same stream.
+ */
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
+
+/*
+ * w4a16_gemm -- Y = X . W^T with W^ dequantized on the fly from the packed
+ * layout (page 3 section 1.2: dequantize fused into the GEMM; page 5 section
+ * 2.2: x^ = (q - zp) * s).
+ *   X        bf16 [M][K] activations, already divided by the smoothing vector
+ *            when one was folded into W (page 3 section 5.3).
+ *   M, N, K  M >= 1, N >= 1, K % group == 0, K >= group.
+ *   qweight, scales, qzeros, group, mode: as produced by w4_quant_pack
+ *            (qzeros NULL in W4_SYM mode).
+ *   Y        out, bf16 [M][N].
+ *   workspace, workspace_bytes: device scratch of at least
+ *            w4a16_workspace_bytes(M, N, K, group) bytes (may be NULL when
+ *            that is 0); 256-byte aligned.
+ * Paths: M <= 8 runs the register GEMV (mma.sync from dequantized registers);
+ * larger M runs the tcgen05 kernel (dequantized weights in tensor memory,
+ * activations in shared memory, fp32 accumulation in tensor memory).
+ */
+w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                     const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
+                     void *workspace, size_t workspace_bytes, w4_stream_t stream);
+
+/* Text for a status code; never NULL. */
+const char *w4_status_string(int status);
+
+/* W4_LAYOUT_VERSION of the library that was loaded. */
+int w4_layout_version(void);
+
+/*
+ * w4_device_error -- read and clear the library's device-side error word.
+ * Kernels that wait on barriers give every wait an iteration limit; a wait
+ * that runs out records a nonzero code here and the kernel returns early
+ * instead of hanging.  This call synchronizes the device.  *code receives 0
+ * when no wait has run out since the last call.
+ */
+w4_status w4_device_error(int *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_H */

@@ -1,0 +1,111 @@
+"""The C ABI: the library loads without a GPU, exports every function that
+include/w4.h declares, and rejects malformed calls on the host before anything
+is launched (so these run on a CPU-only machine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "w4.h")
+
+
+@pytest.fixture(scope="module")
+def w4():
+    from bit_gemm_quant_b200 import build
+    build.build()
+    import bit_gemm_quant_b200 as w4
+    w4.lib()
+    return w4
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("w4_quant_pack", "w4a16_gemm", "w4a16_workspace_bytes", "w4_status_string",
+              "w4_layout_version", "w4_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(w4):
+    L = ctypes.CDLL(w4._LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_layout_version_matches_header(w4):
+    m = re.search(r"#define\s+W4_LAYOUT_VERSION\s+(\d+)", open(HEADER).read())
+    assert w4.w4_layout_version() == int(m.group(1))
+
+
+def test_status_strings(w4):
+    for st in range(4):
+        assert w4.w4_status_string(st).startswith("W4_")
+    assert w4.w4_status_string(99) == "unknown w4 status"
+
+
+FAKE = 1 << 20          # 16-byte aligned fake device addresses: never dereferenced,
+P = ctypes.c_void_p     # every call below is rejected during host-side validation
+
+
+def qp(w4, W=FAKE, N=16, K=256, g=128, mode=0, s=None, q=FAKE, sc=FAKE, z=None):
+    return w4.w4_quant_pack(P(W) if W else None, N, K, g, mode, P(s) if s else None, P(q) if q else None,
+                            P(sc) if sc else None, P(z) if z else None, None)
+
+
+def test_quant_pack_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    assert qp(w4, W=0) == E
+    assert qp(w4, q=0) == E
+    assert qp(w4, sc=0) == E
+    assert qp(w4, N=0) == E                      # empty input
+    assert qp(w4, N=-3) == E
+    assert qp(w4, K=0) == E
+    assert qp(w4, K=200) == E                    # K % g != 0
+    assert qp(w4, g=16) == E and qp(w4, g=256) == E and qp(w4, g=96) == E
+    assert qp(w4, mode=2) == E
+    assert qp(w4, mode=1, z=None) == E           # asymmetric needs qzeros
+    assert qp(w4, mode=0, z=FAKE) == E           # symmetric must not get qzeros
+    assert qp(w4, W=FAKE + 2) == E               # misaligned bf16 input
+    assert qp(w4, q=FAKE + 4) == E
+    assert qp(w4, s=FAKE + 4) == E
+    assert qp(w4, sc=FAKE + 1) == E
+    assert qp(w4, mode=1, z=FAKE + 2) == E
+    assert qp(w4, N=1 << 40, K=1 << 30) == E     # N*K overflows int64
+
+
+def mm(w4, X=FAKE, M=1, N=16, K=256, q=FAKE, sc=FAKE, z=None, g=128, mode=0, Y=FAKE, ws=None, wsb=0):
+    return w4.w4a16_gemm(P(X) if X else None, M, N, K, P(q) if q else None, P(sc) if sc else None,
+                         P(z) if z else None, g, mode, P(Y) if Y else None, P(ws) if ws else None, wsb, None)
+
+
+def test_gemm_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    assert mm(w4, X=0) == E
+    assert mm(w4, Y=0) == E
+    assert mm(w4, q=0) == E
+    assert mm(w4, sc=0) == E
+    assert mm(w4, M=0) == E                      # empty batch
+    assert mm(w4, N=0) == E
+    assert mm(w4, K=64) == E                     # K < g
+    assert mm(w4, K=300) == E
+    assert mm(w4, g=8) == E
+    assert mm(w4, mode=1) == E                   # asymmetric without qzeros
+    assert mm(w4, mode=0, z=FAKE) == E
+    assert mm(w4, X=FAKE + 8) == E
+    assert mm(w4, q=FAKE + 4) == E
+    assert mm(w4, Y=FAKE + 1) == E
+
+
+def test_workspace_query_is_host_only(w4):
+    for M in (1, 4, 8, 16, 32, 512, 8192):
+        assert w4.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
+    assert w4.w4a16_workspace_bytes(1, 4096, 4096, 128) == 0

@@ -1,0 +1,59 @@
+"""Host-side logic of bench.py: argument defaults, the work accounting, and
+the max-over-ranks timing on two gloo ranks (CPU only)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from bit_gemm_quant_b200 import roofline
+
+
+def test_defaults_and_workloads():
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.impl == "w4" and a.workload == "decode" and a.warmup >= 3
+    keys = [k for k, _ in bench.problems_for("decode")]
+    assert len(keys) == 3 and len(set(keys)) == 3
+    assert {k for k, _ in bench.problems_for("prefill")} == {"W"}
+
+
+def test_algorithmic_bytes():
+    # decode N=4096, K=4096, asym g=128: codes 8 MiB, 32 groups/row of fp16 scales, 4 zp words/row
+    assert roofline.packed_bytes(4096, 4096, 128, 1) == 4096 * 2048 + 4096 * 64 + 4096 * 16
+    assert roofline.gemm_bytes(1, 4096, 4096, 128, 1) == 8732672
+    assert roofline.gemm_flops(2048, 14336, 4096) == 2 * 2048 * 14336 * 4096
+    assert roofline.quant_pack_bytes(28672, 8192, 128, 0) == 2 * 28672 * 8192 + 28672 * 4096 + 2 * 28672 * 64
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    ms, units = bench.aggregate(10.0 + 5 * rank, 100 * (rank + 1))
+    bench.barrier()
+    q.put((rank, ms, units))
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms, units in res:
+        assert ms == 15.0 and units == 300.0
