@@ -482,19 +482,19 @@ def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps):
     hW = {k: pin(host_W[k][0]) for k in keys}
     hX = {n: pin(v[0]) for n, v in host_X.items()}
     hs = {k: (torch.from_numpy(host_s[k]).pin_memory() if host_s[k] is not None else None) for k in keys}
-    outs = {}
+    outs_q, outs_y = {}, {}
     h2d = sum(hW[k].numel() * 2 + (hs[k].numel() * 4 if hs[k] is not None else 0) for k in keys) + \
         sum(x.numel() * 2 for x in hX.values())
     d2h = 0
     for k in keys:
         p = qp[k]
         qs, ss, zs = w4.packed_shapes(p.N, p.K, p.group)
-        outs[k] = (torch.empty(qs, dtype=torch.int32).pin_memory(), torch.empty(ss, dtype=torch.float16).pin_memory(),
-                   torch.empty(zs, dtype=torch.int32).pin_memory() if p.mode == 1 else None)
-        d2h += sum(t.numel() * t.element_size() for t in outs[k] if t is not None)
+        outs_q[k] = (torch.empty(qs, dtype=torch.int32).pin_memory(), torch.empty(ss, dtype=torch.float16).pin_memory(),
+                     torch.empty(zs, dtype=torch.int32).pin_memory() if p.mode == 1 else None)
+        d2h += sum(t.numel() * t.element_size() for t in outs_q[k] if t is not None)
     for key, p in plist:
         if p.M > 0:
-            outs[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
+            outs_y[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
             d2h += p.M * p.N * 2
     work = sum(roofline.quant_pack_bytes(qp[k].N, qp[k].K, qp[k].group, qp[k].mode, qp[k].smooth) for k in keys) + \
         sum(roofline.gemm_bytes(p.M, p.N, p.K, p.group, p.mode) for _, p in plist if p.M > 0)
@@ -506,14 +506,14 @@ def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps):
             Wd = hW[k].to(device, non_blocking=True).view(torch.bfloat16)
             sd = hs[k].to(device, non_blocking=True) if hs[k] is not None else None
             q, sc, z = w4.quant_pack(Wd, p.group, p.mode, s=sd)
-            for t_h, t_d in zip(outs[k], (q, sc, z)):
+            for t_h, t_d in zip(outs_q[k], (q, sc, z)):
                 if t_h is not None:
                     t_h.copy_(t_d, non_blocking=True)
             for key, pp in plist:
                 if key == k and pp.M > 0:
                     Xd = hX[pp.name].to(device, non_blocking=True).view(torch.bfloat16)
                     Y = w4.gemm(Xd, q, sc, z, pp.group, pp.mode, N=pp.N)
-                    outs[pp.name].copy_(Y, non_blocking=True)
+                    outs_y[pp.name].copy_(Y, non_blocking=True)
 
     for _ in range(2):
         one()

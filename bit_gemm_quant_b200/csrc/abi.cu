@@ -38,7 +38,7 @@ w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode
     if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
     if (N < 1 || K < 8 || K % group != 0 || !fits(N, K)) return W4_ERR_INVALID_ARG;
     if ((mode == W4_ASYM) != (qzeros != nullptr)) return W4_ERR_INVALID_ARG;
-    if (!aligned(W, 16) || !aligned(qweight, 16) || !aligned(scales, 2)) return W4_ERR_INVALID_ARG;
+    if (!aligned(W, 32) || !aligned(qweight, 16) || !aligned(scales, 2)) return W4_ERR_INVALID_ARG;
     if (s && !aligned(s, 16)) return W4_ERR_INVALID_ARG;
     if (qzeros && !aligned(qzeros, 4)) return W4_ERR_INVALID_ARG;
     const cudaError_t e =
@@ -48,8 +48,9 @@ w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode
 
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group)
 {
-    (void)M; (void)N; (void)K; (void)group;
-    return 0;
+    (void)group;
+    if (M <= 8 || M < 1 || N < 1 || K < 1) return 0;
+    return w4::tc_workspace_bytes(M, N, K);
 }
 
 w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
@@ -67,12 +68,15 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
     const size_t need = w4a16_workspace_bytes(M, N, K, group);
     if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256))))
         return W4_ERR_INVALID_ARG;
-    if (N > (int64_t)INT32_MAX * 16) return W4_ERR_UNSUPPORTED;
     cudaError_t e;
     if (M <= 8) {
+        if (N > INT32_MAX - 16 || K > INT32_MAX) return W4_ERR_UNSUPPORTED;
         e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, Y, (cudaStream_t)stream);
     } else {
-        return W4_ERR_UNSUPPORTED;
+        // tensor-core path: 32-bit indices, TMA extents
+        if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || M * K > INT32_MAX || (int64_t)N * K / 8 > INT32_MAX * 4LL)
+            return W4_ERR_UNSUPPORTED;
+        e = w4::launch_gemm_tc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace, (cudaStream_t)stream);
     }
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
@@ -80,7 +84,10 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
 w4_status w4_device_error(int *code)
 {
     if (!code) return W4_ERR_INVALID_ARG;
-    *code = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
+    const int v = w4::read_and_clear_device_error();
+    if (v < 0) return W4_ERR_CUDA;
+    *code = v;
     return W4_OK;
 }
 

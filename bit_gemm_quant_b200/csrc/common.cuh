@@ -21,5 +21,10 @@ cudaError_t launch_quant_pack(const void *W, int64_t N, int64_t K, int group, in
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                         const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                         cudaStream_t stream);
+size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                           const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
+                           cudaStream_t stream);
+int read_and_clear_device_error();
 
 }  // namespace w4

@@ -1,0 +1,614 @@
+// w4a16_gemm, M > 8: the tensor-core path (tcgen05, tensor memory, TMA).
+//
+// Method: page 4 (llm-glossary.tokens-kit.com/terms/quantization-methods/, GPTQ
+// section) notes that large prefill GEMMs are governed by the dequantize /
+// tensor-core path; page 3 (blog.freezetheflame.cc quantization deep dive)
+// section 1.2 fuses dequantization into the GEMM so weights stay 4-bit in
+// HBM, and its section 3.1 sketches Marlin (INT4 unpacked in registers, fed to
+// tensor cores).  Dequantization follows page 5 (ai-infra.cypggs.com
+// .../02-core-ideas) section 2.2, x^ = (q - zp) * s, rounded once to bf16.
+//
+// B200 design.  The MMA computes the transposed tile
+//     D[128 channels, BN tokens] += W^[128 channels, 16 k] . X[BN tokens, 16 k]^T
+// with tcgen05.mma kind::f16 (bf16 in, fp32 accumulate):
+//   * A = the dequantized weights, written by the dequantizing warps straight
+//     into TENSOR MEMORY with tcgen05.st (lane = output channel, 32-bit column
+//     c of a stage = the bf16 pair (2c, 2c+1) of a 64-wide k-block).  The
+//     weights never touch shared memory, which leaves the shared-memory
+//     bandwidth to the activation operand;
+//   * B = the activations, a [BN tokens x 64 k] bf16 box per k-block, brought
+//     into shared memory by TMA with the 128-byte swizzle the UMMA descriptor
+//     expects (K-major, 8-row atoms of 1024 bytes);
+//   * D lives in tensor memory (BN fp32 columns); the epilogue reads it with
+//     tcgen05.ld, one channel per lane, so a warp writes 32 consecutive
+//     channels of one token (64 contiguous bytes of Y).
+// Warp roles (320 threads): warp 0 issues the TMA loads, warp 1 allocates
+// tensor memory and one of its threads issues the MMAs, warps 2..9 dequantize
+// (warp w owns the 32 lanes 32*(w%4).. of tensor memory and every other
+// k-block) and then run the epilogue.  A 4-stage ring couples them with
+// mbarriers: full_b (TMA bytes landed), full_a (4 warps stored their A
+// slice), empty (tcgen05.commit: the MMAs that read the stage are done).
+// Every wait is bounded in time; a wait that runs out records an error code
+// (read by w4_device_error), raises a CTA-wide abort flag, and the CTA drains
+// its own in-flight copies and MMAs, frees its tensor memory and returns.
+//
+// Split-K: when the tile grid is too small for 148 SMs the k-blocks are split
+// across CTAs; each writes an fp32 partial tile to the caller's workspace and
+// the last CTA of a tile (found with an atomic counter) sums the partials in
+// split order, writes Y and re-zeroes the counter.
+#include "common.cuh"
+
+#include <cuda.h>
+
+namespace w4 {
+
+static __device__ int g_device_error;
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kKB = 64;                      // k per block (one 128-byte swizzle row of bf16)
+constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms; no legitimate wait comes near it
+
+enum : int {
+    kErrWaitTma = 0x101, kErrWaitFullA = 0x102, kErrWaitEmptyTma = 0x103, kErrWaitEmptyDeq = 0x104,
+    kErrWaitDone = 0x105, kErrDrain = 0x106
+};
+
+// ---------------------------------------------------------------- PTX ----
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity.  Gives up (returns false)
+// when the CTA's abort flag is raised or after kWaitLimitNs, in which case it
+// records `code` and raises the abort flag.
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int code)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicCAS(&g_device_error, 0, code);
+            return false;
+        }
+    }
+}
+
+// Drain wait: ignores the abort flag, bounded in time only.
+__device__ __noinline__ bool wait_drain(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicCAS(&g_device_error, 0, kErrDrain);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]^T, one 128 x BN x 16 step.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Dequantization constants of one (channel, group): s_hi = bf16_rne(s16),
+// s_lo = s16 - s_hi (exact, <= 3 significant bits), Z = 128 + zp, each
+// duplicated into both halves of a bf16x2.
+struct GroupConst {
+    uint32_t shi, slo, z;
+};
+
+__device__ __forceinline__ GroupConst group_const(unsigned short s16bits, uint32_t zp)
+{
+    const float sf = __half2float(__ushort_as_half(s16bits));
+    const __nv_bfloat16 hi = __float2bfloat16_rn(sf);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(sf - __bfloat162float(hi));
+    const uint32_t h = __bfloat16_as_ushort(hi), l = __bfloat16_as_ushort(lo);
+    GroupConst gc;
+    gc.shi = h | (h << 16);
+    gc.slo = l | (l << 16);
+    gc.z = 0x43004300u | (zp << 16) | zp;
+    return gc;
+}
+
+// w^ for the adjacent elements (8c+2j, 8c+2j+1) held by packed word q:
+// (128+u) - (128+zp) is exact, D*s_lo is exact, and fma(D, s_hi, D*s_lo)
+// rounds the exact product D*s16 once to bf16.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupConst &gc)
+{
+    const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+    const uint32_t D = bf2_sub(v, gc.z);
+    return bf2_fma(D, gc.shi, bf2_mul(D, gc.slo));
+}
+
+// UMMA shared-memory descriptor of a K-major operand stored with the 128-byte
+// swizzle: 8-row atoms of 1024 bytes (stride byte offset 1024), leading byte
+// offset 16 (unused for this layout), descriptor version 1, layout type 2.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+template <int BN>
+struct TcCfg {
+    static constexpr int kACol0 = BN;                                   // A stages follow the BN fp32 accumulator columns
+    static constexpr int kCols = (BN + kStages * 32 <= 256) ? 256 : 512; // tensor-memory allocation
+    static constexpr int kStageBytes = BN * 128;                        // activation box bytes
+    static constexpr int kMinBlocks = (BN == 256) ? 1 : 2;
+    // kind::f16, fp32 D, bf16 A and B, both K-major, N = BN, M = 128
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+};
+
+struct SlotData {
+    uint4 w0, w1;
+    unsigned short s0, s1;
+    uint32_t z0, z1;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, TcCfg<BN>::kMinBlocks)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, int group_log2, int asym,
+               const uint4 *__restrict__ qweight, const unsigned short *__restrict__ scales,
+               const uint32_t *__restrict__ qzeros, __nv_bfloat16 *__restrict__ Y, float *__restrict__ partial,
+               unsigned *__restrict__ counters, int splits, int kb_per_split)
+{
+    using C = TcCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sB = smem;                                               // kStages x BN x 128 bytes
+    uint64_t *full_b = (uint64_t *)(smem + kStages * C::kStageBytes);
+    uint64_t *full_a = full_b + kStages;
+    uint64_t *empty = full_a + kStages;
+    uint64_t *done = empty + kStages;
+    uint32_t *tmem_slot = (uint32_t *)(done + 1);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+    int *last_flag = (int *)(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN, split = blockIdx.z;
+    const int KQ = K >> 5;                                            // 16-byte code chunks per channel
+    const int kb_total = (K + kKB - 1) / kKB;
+    const int kb_begin = split * kb_per_split;
+    const int nkb = min(kb_total, kb_begin + kb_per_split) - kb_begin;
+    const int NG = K >> group_log2, ZW = (NG + 7) >> 3;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_b[s], 1);
+            mbar_init(&full_a[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, C::kCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_x) : "memory");
+            int issued = 0;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyTma)) break;
+                mbar_arrive_expect_tx(&full_b[s], C::kStageBytes);
+                tma_load_2d(sB + s * C::kStageBytes, &tmap_x, &full_b[s], (kb_begin + i) * kKB, m0);
+                ++issued;
+            }
+            // drain: every issued copy must have landed before the CTA may exit
+            for (int i = max(0, issued - kStages); i < issued; ++i)
+                wait_drain(&full_b[i % kStages], (i / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ---
+        if (lane == 0) {
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!wait_bounded(&full_a[s], ph, abort_flag, kErrWaitFullA)) break;
+                if (!wait_bounded(&full_b[s], ph, abort_flag, kErrWaitTma)) break;
+                tc_fence_after();
+                const uint64_t bdesc = desc_k_sw128(smem_u32(sB + s * C::kStageBytes));
+#pragma unroll
+                for (int kk = 0; kk < kKB / 16; ++kk)
+                    mma_ts(tmem, tmem + C::kACol0 + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2), C::kIdesc,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&empty[s]);
+            }
+            mma_commit(done);
+            wait_drain(done, 0);   // no MMA may still be running when tensor memory is freed
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------- dequantize, then epilogue --
+        const int q = warp & 3;                      // tensor-memory lane quarter of this warp
+        const int h = (warp - 2) >> 2;               // k-block parity handled by this warp
+        const int r = 32 * q + lane;
+        const int n = n0 + r;
+        const bool okn = n < N;
+        const uint4 *qrow = qweight + (size_t)(okn ? n : 0) * KQ;
+        const unsigned short *srow = scales + (size_t)(okn ? n : 0) * NG;
+        const uint32_t *zrow = qzeros + (size_t)(okn ? n : 0) * ZW;
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+
+        constexpr int D = 4;                         // k-blocks prefetched per thread
+        SlotData buf[D];
+        auto fetch = [&](int i, SlotData &sd) {
+            const int kq = (kb_begin + i) * 2;       // first 16-byte chunk of this k-block
+            const bool ok0 = okn, ok1 = okn && (kq + 1 < KQ);
+            sd.w0 = ok0 ? ld_stream(qrow + kq) : make_uint4(0u, 0u, 0u, 0u);
+            sd.w1 = ok1 ? ld_stream(qrow + kq + 1) : make_uint4(0u, 0u, 0u, 0u);
+            const int j0 = (kq * 32) >> group_log2, j1 = ((kq + 1) * 32) >> group_log2;
+            sd.s0 = ok0 ? __ldg(srow + j0) : (unsigned short)0;
+            sd.s1 = ok1 ? __ldg(srow + j1) : (unsigned short)0;
+            if (asym) {
+                sd.z0 = ok0 ? (__ldg(zrow + (j0 >> 3)) >> (4 * (j0 & 7))) & 0xFu : 0u;
+                sd.z1 = ok1 ? (__ldg(zrow + (j1 >> 3)) >> (4 * (j1 & 7))) & 0xFu : 0u;
+            } else {
+                sd.z0 = sd.z1 = 8u;
+            }
+        };
+#pragma unroll
+        for (int d = 0; d < D; ++d)
+            if (h + 2 * d < nkb) fetch(h + 2 * d, buf[d]);
+
+        bool ok = true;
+        for (int i0 = h; i0 < nkb && ok; i0 += 2 * D) {
+#pragma unroll
+            for (int d = 0; d < D; ++d) {
+                const int i = i0 + 2 * d;
+                if (i >= nkb || !ok) break;
+                uint32_t v[32];
+                const GroupConst c0 = group_const(buf[d].s0, buf[d].z0);
+                const GroupConst c1 = group_const(buf[d].s1, buf[d].z1);
+                const uint32_t wa[4] = {buf[d].w0.x, buf[d].w0.y, buf[d].w0.z, buf[d].w0.w};
+                const uint32_t wb[4] = {buf[d].w1.x, buf[d].w1.y, buf[d].w1.z, buf[d].w1.w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        v[4 * w + j] = dequant_pair(wa[w], j, c0);
+                        v[16 + 4 * w + j] = dequant_pair(wb[w], j, c1);
+                    }
+                if (i + 2 * D < nkb) fetch(i + 2 * D, buf[d]);
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                if (!__all_sync(0xffffffffu, wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyDeq))) {
+                    ok = false;
+                    break;
+                }
+                tmem_st32(lane_addr + C::kACol0 + s * 32, v);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_a[s]);
+            }
+        }
+
+        // ---- epilogue: accumulator -> Y (or fp32 partials) ----
+        const bool have = __all_sync(0xffffffffu, ok && wait_bounded(done, 0, abort_flag, kErrWaitDone));
+        tc_fence_after();
+        constexpr int HALF = BN / 2;                  // columns per warp of a lane quarter
+        const int cbeg = h * HALF;
+        if (have) {
+            for (int c = 0; c < HALF; c += 8) {
+                float acc[8];
+                tmem_ld8(lane_addr + cbeg + c, acc);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + cbeg + c + j;
+                    if (okn && m < M) {
+                        if (splits == 1) Y[(size_t)m * N + n] = __float2bfloat16_rn(acc[j]);
+                        else partial[((size_t)split * M + m) * N + n] = acc[j];
+                    }
+                }
+            }
+        }
+        if (splits > 1) {
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (threadIdx.x == 64) {
+                const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
+                const unsigned prev = atomicAdd(&counters[tile], 1u);
+                *last_flag = (prev == (unsigned)splits - 1) ? 1 : 0;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (*(volatile int *)last_flag) {
+                __threadfence();
+                for (int c = 0; c < HALF; ++c) {
+                    const int m = m0 + cbeg + c;
+                    if (okn && m < M) {
+                        float sum = 0.f;
+                        for (int sp = 0; sp < splits; ++sp) sum += __ldcg(partial + ((size_t)sp * M + m) * N + n);
+                        Y[(size_t)m * N + n] = __float2bfloat16_rn(sum);
+                    }
+                }
+                if (threadIdx.x == 64) counters[blockIdx.y * gridDim.x + blockIdx.x] = 0u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::kCols);
+}
+
+// ----------------------------------------------------------------- host --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+struct TcPlan {
+    int BN = 0, splits = 1, kb_per_split = 0, m_tiles = 0, n_tiles = 0;
+    size_t ws_bytes = 0;
+};
+
+int pick_bn(int64_t M)
+{
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+TcPlan plan_tc(int64_t M, int64_t N, int64_t K)
+{
+    TcPlan p;
+    p.BN = pick_bn(M);
+    p.m_tiles = (int)((M + p.BN - 1) / p.BN);
+    p.n_tiles = (int)((N + 127) / 128);
+    const int kb_total = (int)((K + kKB - 1) / kKB);
+    const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
+    const int per_sm = (p.BN == 256) ? 1 : 2;
+    const int64_t slots = (int64_t)kNumSMs * per_sm;
+    int best = 1;
+    if (p.BN <= 64 && tiles < 4 * slots) {
+        // skinny, bandwidth-bound: split k so the grid fills whole waves of the SMs
+        double best_eff = -1.0;
+        for (int s = 1; s <= 8 && kb_total / s >= 4; ++s) {
+            const int64_t ctas = tiles * s;
+            const int64_t waves = (ctas + slots - 1) / slots;
+            const double eff = (double)ctas / (double)(waves * slots);
+            if (eff > best_eff + 0.02) { best_eff = eff; best = s; }
+        }
+    }
+    p.kb_per_split = (kb_total + best - 1) / best;
+    p.splits = (kb_total + p.kb_per_split - 1) / p.kb_per_split;
+    if (p.splits > 1) {
+        const size_t part = (size_t)p.splits * M * N * sizeof(float);
+        const size_t part_al = (part + 255) & ~(size_t)255;
+        p.ws_bytes = part_al + (size_t)tiles * sizeof(unsigned);
+    }
+    return p;
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap &map, const TcPlan &p, int M, int N, int K, int glog2, int asym,
+                      const uint32_t *qweight, const void *scales, const uint32_t *qzeros, void *Y, void *ws,
+                      cudaStream_t stream)
+{
+    using C = TcCfg<BN>;
+    size_t smem = 1024 + kStages * C::kStageBytes + 256;
+    if (C::kMinBlocks == 2 && smem < 80 * 1024) smem = 80 * 1024;   // at most 2 CTAs share an SM's tensor memory
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    float *partial = nullptr;
+    unsigned *counters = nullptr;
+    if (p.splits > 1) {
+        const size_t part = (size_t)p.splits * M * N * sizeof(float);
+        partial = (float *)ws;
+        counters = (unsigned *)((uint8_t *)ws + ((part + 255) & ~(size_t)255));
+    }
+    dim3 grid(p.n_tiles, p.m_tiles, p.splits);
+    gemm_tc_kernel<BN><<<grid, kThreads, smem, stream>>>(
+        map, M, N, K, glog2, asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
+        (__nv_bfloat16 *)Y, partial, counters, p.splits, p.kb_per_split);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K) { return plan_tc(M, N, K).ws_bytes; }
+
+cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                           const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
+                           cudaStream_t stream)
+{
+    const TcPlan p = plan_tc(M, N, K);
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kKB, (cuuint32_t)p.BN};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), gdim, gstride, box,
+                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const int glog2 = group == 32 ? 5 : group == 64 ? 6 : 7;
+    const int asym = mode == W4_ASYM;
+    switch (p.BN) {
+    case 16: return launch_bn<16>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 32: return launch_bn<32>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 64: return launch_bn<64>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 128: return launch_bn<128>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    default: return launch_bn<256>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    }
+}
+
+int read_and_clear_device_error()
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+    const int zero = 0;
+    if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+    return v;
+}
+
+}  // namespace w4

@@ -11,9 +11,13 @@
 // .../02-core-ideas) section 2.2, x^ = (q - zp) * s, rounded once to bf16.
 //
 // Design (HBM-bound: 0.5 B of codes + 1/64 B of scale per weight at g = 128):
-//   * a CTA owns 16 output channels and all of K; its 8 warps split K into
-//     512-wide super-chunks (warp w takes super-chunks w, w+8, ...), and sum
-//     their partial tiles in shared memory at the end (no global scratch);
+//   * a tile is 16 output channels and all of K; a CTA loops over the tiles
+//     blockIdx.x, blockIdx.x + gridDim.x, ... (two CTAs per SM, every CTA the
+//     same number of tiles); its 8 warps split K into 512-wide super-chunks
+//     (warp w takes super-chunks w, w+8, ...) and sum their partial tiles in
+//     double-buffered shared memory after the last super-chunk of each tile
+//     (no global scratch); each warp loads its next work item before it
+//     computes the current one;
 //   * lane (g, t) = (lane/4, lane%4) of a warp loads, for channels g and g+8,
 //     the 64 contiguous bytes (128 codes) at k = 512*sc + 128*t: all of its
 //     loads are issued before any arithmetic (8 x 16 B per lane);
@@ -106,57 +110,75 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupC
 
 constexpr int kWarps = 8;
 
+// A warp's work item is one 512-wide super-chunk of K for the 16 channels of
+// a tile: 4 x 16 bytes of codes per lane for each of its two channels.
+struct Item {
+    uint4 a[4], b[4];
+};
+
 template <int G, int MODE>
-__global__ void __launch_bounds__(kWarps * 32)
-gemv_kernel(const uint4 *__restrict__ X, int M, int64_t N, int64_t K, const uint4 *__restrict__ qweight,
+__global__ void __launch_bounds__(kWarps * 32, 2)
+gemv_kernel(const uint4 *__restrict__ X, int M, int N, int K, const uint4 *__restrict__ qweight,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
             __nv_bfloat16 *__restrict__ Y)
 {
-    constexpr int QPG = G / 32;                  // 32-code chunks per group
-    __shared__ float red[kWarps][32][4];
+    constexpr int QPG = G / 32;                  // 16-byte code chunks per group
+    __shared__ float red[2][kWarps][32][4];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int64_t rowA = (int64_t)blockIdx.x * 16 + g, rowB = rowA + 8;
-    const bool okA = rowA < N, okB = rowB < N;
-    const int64_t KQ = K >> 5;                   // 16-byte code chunks per channel
-    const int64_t NG = K / G, ZW = (NG + 7) >> 3;
+    const int KQ = K >> 5;                       // 16-byte code chunks per channel
+    const int NG = K / G, ZW = (NG + 7) >> 3;
+    const int ntiles = (N + 15) >> 4;
+    const int nsc = (KQ + 15) >> 4;              // 512-wide super-chunks per channel
+    const int per_warp = (nsc + kWarps - 1) / kWarps;
+    const int my_tiles = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int items = my_tiles * per_warp;
     const bool has_x = g < M;
-    const uint4 *xrow = X + (int64_t)(has_x ? g : 0) * (K >> 3);
+    const uint4 *xrow = X + (size_t)(has_x ? g : 0) * (K >> 3);
 
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-
-    for (int64_t sc = warp; sc * 16 < KQ; sc += kWarps) {
-        const int64_t q0 = sc * 16 + t * 4;      // first chunk of this lane
-        uint4 qa[4], qb[4];
+    auto fetch = [&](int it, Item &d) {
+        const int tile = (int)blockIdx.x + (it / per_warp) * (int)gridDim.x;
+        const int q0 = (warp + kWarps * (it % per_warp)) * 16 + t * 4;
+        const int rA = tile * 16 + g, rB = rA + 8;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const bool ok = q0 + i < KQ;
-            qa[i] = (ok && okA) ? ld_stream(qweight + rowA * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
-            qb[i] = (ok && okB) ? ld_stream(qweight + rowB * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+            d.a[i] = (ok && rA < N) ? ld_stream(qweight + (size_t)rA * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+            d.b[i] = (ok && rB < N) ? ld_stream(qweight + (size_t)rB * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
         }
+    };
+
+    Item cur, nxt;
+    if (items > 0) fetch(0, cur);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int it = 0; it < items; ++it) {
+        if (it + 1 < items) fetch(it + 1, nxt);
+        const int tile = (int)blockIdx.x + (it / per_warp) * (int)gridDim.x;
+        const int q0 = (warp + kWarps * (it % per_warp)) * 16 + t * 4;
+        const int rA = tile * 16 + g, rB = rA + 8;
+        const bool okA = rA < N, okB = rB < N;
         GroupConst ca, cb;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int64_t qi = q0 + i;
+            const int qi = q0 + i;
             const bool ok = qi < KQ;
-            const int64_t k = qi * 32;
             if (i % QPG == 0) {
-                const int64_t j = ok ? k / G : 0;
-                int za = 8, zb = 8;
+                const int j = ok ? (qi * 32) / G : 0;
+                uint32_t za = 8u, zb = 8u;
                 if (MODE == W4_ASYM) {
-                    za = okA ? (int)((__ldg(qzeros + rowA * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu) : 0;
-                    zb = okB ? (int)((__ldg(qzeros + rowB * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu) : 0;
+                    za = okA ? (__ldg(qzeros + (size_t)rA * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
+                    zb = okB ? (__ldg(qzeros + (size_t)rB * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
                 }
-                ca = group_const(okA ? __ldg(scales + rowA * NG + j) : (unsigned short)0, za);
-                cb = group_const(okB ? __ldg(scales + rowB * NG + j) : (unsigned short)0, zb);
+                ca = group_const(okA ? __ldg(scales + (size_t)rA * NG + j) : (unsigned short)0, (int)za);
+                cb = group_const(okB ? __ldg(scales + (size_t)rB * NG + j) : (unsigned short)0, (int)zb);
             }
             uint4 xv[4];
 #pragma unroll
             for (int w = 0; w < 4; ++w)
-                xv[w] = (has_x && ok) ? __ldg(xrow + (k >> 3) + w) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t wa[4] = {qa[i].x, qa[i].y, qa[i].z, qa[i].w};
-            const uint32_t wb[4] = {qb[i].x, qb[i].y, qb[i].z, qb[i].w};
+                xv[w] = (has_x && ok) ? __ldg(xrow + qi * 4 + w) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t wa[4] = {cur.a[i].x, cur.a[i].y, cur.a[i].z, cur.a[i].w};
+            const uint32_t wb[4] = {cur.b[i].x, cur.b[i].y, cur.b[i].z, cur.b[i].w};
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const uint32_t a0 = dequant_pair(wa[w], 0, ca), a1 = dequant_pair(wa[w], 1, ca);
@@ -167,24 +189,28 @@ gemv_kernel(const uint4 *__restrict__ X, int M, int64_t N, int64_t K, const uint
                 mma_bf16_16816(acc, a2, b2, a3, b3, xv[w].z, xv[w].w);
             }
         }
-    }
-
-    red[warp][lane][0] = acc[0];
-    red[warp][lane][1] = acc[1];
-    red[warp][lane][2] = acc[2];
-    red[warp][lane][3] = acc[3];
-    __syncthreads();
-    if (warp == 0) {
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        if (it % per_warp == per_warp - 1) {     // last super-chunk of this tile: reduce the 8 warps
+            const int buf = (it / per_warp) & 1;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
+            for (int i = 0; i < 4; ++i) {
+                red[buf][warp][lane][i] = acc[i];
+                acc[i] = 0.f;
+            }
+            __syncthreads();
+            if (warp == 0) {
+                float sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) s[i] += red[w][lane][i];
-        const int m0 = 2 * t, m1 = 2 * t + 1;    // tokens of c0/c2 and c1/c3
-        if (okA && m0 < M) Y[(int64_t)m0 * N + rowA] = __float2bfloat16_rn(s[0]);
-        if (okA && m1 < M) Y[(int64_t)m1 * N + rowA] = __float2bfloat16_rn(s[1]);
-        if (okB && m0 < M) Y[(int64_t)m0 * N + rowB] = __float2bfloat16_rn(s[2]);
-        if (okB && m1 < M) Y[(int64_t)m1 * N + rowB] = __float2bfloat16_rn(s[3]);
+                for (int w = 0; w < kWarps; ++w)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sm[i] += red[buf][w][lane][i];
+                const int m0 = 2 * t, m1 = 2 * t + 1;   // tokens of c0/c2 and c1/c3
+                if (okA && m0 < M) Y[(size_t)m0 * N + rA] = __float2bfloat16_rn(sm[0]);
+                if (okA && m1 < M) Y[(size_t)m1 * N + rA] = __float2bfloat16_rn(sm[1]);
+                if (okB && m0 < M) Y[(size_t)m0 * N + rB] = __float2bfloat16_rn(sm[2]);
+                if (okB && m1 < M) Y[(size_t)m1 * N + rB] = __float2bfloat16_rn(sm[3]);
+            }
+        }
+        cur = nxt;
     }
 }
 
@@ -192,9 +218,13 @@ template <int G, int MODE>
 cudaError_t launch_g_mode(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                           const void *scales, const uint32_t *qzeros, void *Y, cudaStream_t stream)
 {
-    const int64_t blocks = (N + 15) / 16;
+    // as many CTAs as two per SM allow, rounded so that every CTA gets the same number of tiles
+    const int64_t ntiles = (N + 15) / 16;
+    const int64_t slots = (int64_t)kNumSMs * 2;
+    const int64_t per_cta = (ntiles + slots - 1) / slots;
+    const int64_t blocks = (ntiles + per_cta - 1) / per_cta;
     gemv_kernel<G, MODE><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-        (const uint4 *)X, (int)M, N, K, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
+        (const uint4 *)X, (int)M, (int)N, (int)K, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
         (__nv_bfloat16 *)Y);
     return cudaGetLastError();
 }

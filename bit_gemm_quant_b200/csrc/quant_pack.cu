@@ -7,182 +7,195 @@
 // (blog.freezetheflame.cc quantization deep dive) section 5.3 the offline fold
 // W * s.  The exact arithmetic is spelled out in include/w4.h.
 //
-// Design (HBM-bound stream: 2 B read + 0.5 B written per weight):
-//   * one warp per row at a time (grid-stride over rows); a lane owns 8
-//     consecutive weights (one 16-byte load), so a group of g weights is g/8
-//     adjacent lanes and its amax / min / max is a butterfly of
-//     __shfl_xor_sync over those lanes;
-//   * a batch is 4 loads per lane (1024 weights per warp) issued before any
-//     arithmetic, so every warp keeps 2 KB in flight;
-//   * each lane packs its 8 codes into one 32-bit word (even elements in the
-//     low half-word), so a warp stores 128 contiguous bytes per iteration;
-//     zero-points of 8 groups are OR-reduced across the warp with
-//     __reduce_or_sync and stored once per word;
-//   * per element the code is rint(w'/s16) with IEEE semantics: the quotient
-//     is first approximated as w' * rcp(s16); when that approximation is
-//     further than 2^-10 from every half-integer its rounding cannot differ
-//     from that of the exact quotient (the approximation error is below
-//     2^-18), so the code is read from the approximation with a magic-number
-//     add; otherwise the lane recomputes its 8 codes with correctly rounded
-//     division (__fdiv_rn).  Per-group scale and zero-point use __fdiv_rn
-//     directly, so both are bit-identical to the IEEE definitions.
+// Design (HBM-bound stream: 2 B read + about 0.5 B written per weight, a
+// budget of roughly 0.4 warp instructions per weight at full bandwidth):
+//   * one warp per row at a time (grid-stride over rows); a lane owns 32
+//     consecutive weights, which always lie in one group (g = 32, 64, 128 is
+//     1, 2 or 4 lanes), read with two 32-byte loads; the next 1024 weights of
+//     the row are loaded before the current ones are processed;
+//   * group amax / min / max: 32 in-lane comparisons and at most two
+//     __shfl_xor_sync steps; the per-group IEEE divisions (scale and zero
+//     point) and the reciprocal are then amortized over 32 weights per lane;
+//   * per weight the code is rint(w'/s16) with IEEE semantics: the quotient
+//     is approximated as t = w' * rcp(s16); adding the magic constant
+//     1.5*2^23 + zp leaves 0x4B400000 + u in the float's bits.  If every t of
+//     the lane is further than 2^-10 from a half-integer (the approximation
+//     error is below 2^-18) those codes equal the codes of the exact quotient;
+//     otherwise the lane recomputes its 32 codes with correctly rounded
+//     division (__fdiv_rn).  No lower clamp is needed (the group minimum maps
+//     to -zp exactly) and in symmetric mode no clamp at all (|t| <= 7 * (1 +
+//     2^-11)); groups whose fp16 scale saturated or is subnormal take the
+//     exact path;
+//   * packing: with bits(y) = C + u (C's low byte 0), one IMAD y_b*16 + y_a
+//     puts the byte u_a | u_b << 4 in the low byte; three PRMTs assemble the
+//     word (even elements in the low half-word), and each lane stores its 4
+//     words as one 16-byte store (a warp writes 512 contiguous bytes);
+//   * zero-points of 8 groups are OR-reduced with __shfl_xor_sync inside their
+//     8*g/32-lane segment and stored once per word.
 #include "common.cuh"
 
 namespace w4 {
 namespace {
 
-// 1.5 * 2^23: for |t| < 2^22, fl32(t + kMagic) has rint(t) (ties to even) in
-// its low mantissa bits, because the spacing of floats in [2^23, 2^24) is 1.
+// 1.5 * 2^23: for |t| < 2^22, fl32(t + kMagic) has rint(t) in its low mantissa
+// bits, because the spacing of floats in [2^23, 2^24) is 1.
 constexpr float kMagic = 12582912.0f;
 // Quotients closer than 2^-10 to a half-integer take the exact path.
 constexpr float kNearTie = 0.5f - 0.0009765625f;
 
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+__device__ __forceinline__ void ld32(const uint4 *p, uint32_t (&v)[8])
 {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+    asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
                  : "l"(p));
-    return v;
 }
 
-// Bit offset of element e (0..7) inside its packed word: even elements in the
-// low half-word, odd elements in the high half-word.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// One packed word from the magic-added floats of elements 0..7 of an 8-chunk:
+// bytes (e0|e2<<4), (e4|e6<<4), (e1|e3<<4), (e5|e7<<4).
+__device__ __forceinline__ uint32_t pack_word(const float *y)
+{
+    const uint32_t p0 = __float_as_uint(y[2]) * 16u + __float_as_uint(y[0]);
+    const uint32_t p1 = __float_as_uint(y[6]) * 16u + __float_as_uint(y[4]);
+    const uint32_t p2 = __float_as_uint(y[3]) * 16u + __float_as_uint(y[1]);
+    const uint32_t p3 = __float_as_uint(y[7]) * 16u + __float_as_uint(y[5]);
+    return prmt(prmt(p0, p1, 0x0040u), prmt(p2, p3, 0x0040u), 0x5410u);
+}
+
 __host__ __device__ constexpr int nibble_shift(int e) { return (e & 1) ? 16 + 4 * (e >> 1) : 4 * (e >> 1); }
 
 template <int G, int MODE, bool FOLD>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float4 *__restrict__ s,
-                  uint32_t *__restrict__ qweight, unsigned short *__restrict__ scales,
-                  uint32_t *__restrict__ qzeros)
+                  uint4 *__restrict__ qweight, unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros)
 {
-    constexpr int LPG = G / 8;                  // lanes per group
-    constexpr int ZPB = 128 / G;                // zero-point words per 1024-weight batch
+    constexpr int LPG = G / 32;                 // lanes per group
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t KW = K >> 3;                  // packed words (= 16-byte bf16 chunks) per row
+    const int64_t KC = K >> 5;                  // 32-weight chunks per row
     const int64_t NG = K / G;                   // groups per row
     const int64_t ZW = (NG + 7) >> 3;           // zero-point words per row
 
     for (int64_t n = warp0; n < N; n += nwarps) {
-        const uint4 *row = W + n * KW;
-        for (int64_t c0 = 0; c0 < KW; c0 += 128) {
-            uint4 v[4];
-            float4 sa[4], sb[4];
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int64_t c = c0 + it * 32 + lane;
-                if (c < KW) {
-                    v[it] = ld_stream(row + c);
-                    if (FOLD) { sa[it] = __ldg(s + 2 * c); sb[it] = __ldg(s + 2 * c + 1); }
-                } else {
-                    v[it] = make_uint4(0u, 0u, 0u, 0u);
-                    if (FOLD) { sa[it] = make_float4(1.f, 1.f, 1.f, 1.f); sb[it] = sa[it]; }
-                }
+        const uint4 *row = W + n * (K >> 3);    // 8 bf16 per uint4
+        uint32_t cur[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        {
+            const int64_t c = lane;
+            if (c < KC) { ld32(row + 4 * c, *(uint32_t(*)[8])&cur[0]); ld32(row + 4 * c + 2, *(uint32_t(*)[8])&cur[8]); }
+        }
+        for (int64_t c0 = 0; c0 < KC; c0 += 32) {
+            const int64_t c = c0 + lane;        // this lane's chunk
+            const bool valid = c < KC;
+            uint32_t nxt[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            if (c + 32 < KC) {                  // prefetch the next 1024 weights of the row
+                ld32(row + 4 * (c + 32), *(uint32_t(*)[8])&nxt[0]);
+                ld32(row + 4 * (c + 32) + 2, *(uint32_t(*)[8])&nxt[8]);
             }
-            uint32_t zacc[ZPB];
+            float x[32];
 #pragma unroll
-            for (int i = 0; i < ZPB; ++i) zacc[i] = 0u;
-
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int64_t c = c0 + it * 32 + lane;
-                const bool valid = c < KW;
-                float x[8];
-                x[0] = bf16lo_to_f32(v[it].x); x[1] = bf16hi_to_f32(v[it].x);
-                x[2] = bf16lo_to_f32(v[it].y); x[3] = bf16hi_to_f32(v[it].y);
-                x[4] = bf16lo_to_f32(v[it].z); x[5] = bf16hi_to_f32(v[it].z);
-                x[6] = bf16lo_to_f32(v[it].w); x[7] = bf16hi_to_f32(v[it].w);
-                if (FOLD) {   // w' = fl32(w * s[k])
-                    x[0] = __fmul_rn(x[0], sa[it].x); x[1] = __fmul_rn(x[1], sa[it].y);
-                    x[2] = __fmul_rn(x[2], sa[it].z); x[3] = __fmul_rn(x[3], sa[it].w);
-                    x[4] = __fmul_rn(x[4], sb[it].x); x[5] = __fmul_rn(x[5], sb[it].y);
-                    x[6] = __fmul_rn(x[6], sb[it].z); x[7] = __fmul_rn(x[7], sb[it].w);
-                }
-
-                float d, inv, lo, hi;
-                int zp;
-                unsigned short s16;
-                if (MODE == W4_SYM) {
-                    float a = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(x[i]));
-#pragma unroll
-                    for (int off = LPG / 2; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-                    const float s32 = __fdiv_rn(a, 7.0f);
-                    s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
-                    d = __half2float(__ushort_as_half(s16));
-                    inv = (d > 0.f) ? __frcp_rn(d) : 0.f;
-                    zp = 8;
-                    lo = -8.f;
-                    hi = 7.f;
-                } else {
-                    float mn = 0.f, mx = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
-#pragma unroll
-                    for (int off = LPG / 2; off > 0; off >>= 1) {
-                        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                    }
-                    const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-                    s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
-                    d = __half2float(__ushort_as_half(s16));
-                    if (d > 0.f) {
-                        inv = __frcp_rn(d);
-                        zp = (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, d)), 0.f), 15.f);
-                    } else {
-                        inv = 0.f;
-                        zp = 0;
-                    }
-                    lo = (float)(-zp);
-                    hi = (float)(15 - zp);
-                }
-
-                // codes: fast path from the approximate quotient
-                uint32_t word = 0u;
-                bool near_tie = false;
-                const float magic = (MODE == W4_SYM) ? kMagic + 8.0f : kMagic;   // both even
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t v = valid ? cur[i] : 0u;
+                x[2 * i] = bf16lo_to_f32(v);
+                x[2 * i + 1] = bf16hi_to_f32(v);
+            }
+            if (FOLD && valid) {                // w' = fl32(w * s[k])
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float t = fminf(fmaxf(__fmul_rn(x[i], inv), lo), hi);
-                    const float y = __fadd_rn(t, magic);
-                    const float r = __fsub_rn(y, magic);
-                    near_tie |= fabsf(__fsub_rn(t, r)) > kNearTie;
-                    uint32_t u = __float_as_uint(y);
-                    if (MODE == W4_ASYM) u += (uint32_t)zp;
-                    word |= (u & 0xFu) << nibble_shift(i);
+                    const float4 f = __ldg(s + 8 * c + i);
+                    x[4 * i] = __fmul_rn(x[4 * i], f.x);
+                    x[4 * i + 1] = __fmul_rn(x[4 * i + 1], f.y);
+                    x[4 * i + 2] = __fmul_rn(x[4 * i + 2], f.z);
+                    x[4 * i + 3] = __fmul_rn(x[4 * i + 3], f.w);
                 }
-                if (near_tie) {   // exact path: rint of the correctly rounded quotient
-                    word = 0u;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float q = rintf(__fdiv_rn(x[i], d));
-                        int u;
-                        if (MODE == W4_SYM) u = (int)fminf(fmaxf(q, -8.f), 7.f) + 8;
-                        else u = (int)fminf(fmaxf(q + (float)zp, 0.f), 15.f);
-                        word |= (uint32_t)u << nibble_shift(i);
-                    }
-                }
+            }
 
-                const int64_t j = (c * 8) / G;      // group of this lane
-                if (valid) {
-                    qweight[n * KW + c] = word;
-                    if ((lane % LPG) == 0) scales[n * NG + j] = s16;
+            // ---- group statistics, scale and zero-point ----
+            float d, inv, magic, hi = 0.f;
+            int zp;
+            unsigned short s16;
+            bool exact_only;
+            if (MODE == W4_SYM) {
+                float a = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+#pragma unroll
+                for (int off = LPG / 2; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+                const float s32 = __fdiv_rn(a, 7.0f);
+                s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
+                d = __half2float(__ushort_as_half(s16));
+                zp = 8;
+            } else {
+                float mn = 0.f, mx = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
+#pragma unroll
+                for (int off = LPG / 2; off > 0; off >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
                 }
-                if (MODE == W4_ASYM) {
-                    const uint32_t mine = (valid && (lane % LPG) == 0) ? ((uint32_t)zp << (4 * (int)(j & 7))) : 0u;
-                    zacc[(it * 32) / G] |= __reduce_or_sync(0xffffffffu, mine);
+                const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+                s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
+                d = __half2float(__ushort_as_half(s16));
+                zp = (d > 0.f) ? (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, d)), 0.f), 15.f) : 0;
+                hi = (float)(15 - zp);
+            }
+            // the fast path assumes a normal, unsaturated fp16 scale (or a zero one)
+            exact_only = (s16 == 0x7BFF) || (d > 0.f && d < 6.103515625e-05f);
+            inv = (d > 0.f) ? __frcp_rn(d) : 0.f;
+            magic = kMagic + (float)zp;         // exact: 1.5*2^23 + zp < 2^24
+
+            // ---- codes: fast path, one packed word per 8 weights ----
+            uint4 out;
+            uint32_t wd[4];
+            float emax = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float t = __fmul_rn(x[8 * w + i], inv);
+                    if (MODE == W4_ASYM) t = fminf(t, hi);
+                    y[i] = __fadd_rn(t, magic);
+                    emax = fmaxf(emax, fabsf(__fsub_rn(t, __fsub_rn(y[i], magic))));
                 }
+                wd[w] = pack_word(y);
+            }
+            if (!(emax > kNearTie || exact_only)) {
+                out = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            } else {                            // exact path: rint of the correctly rounded quotient
+                uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float q = (d > 0.f) ? rintf(__fdiv_rn(x[i], d)) : 0.f;
+                    int u;
+                    if (MODE == W4_SYM) u = (int)fminf(fmaxf(q, -8.f), 7.f) + 8;
+                    else u = (int)fminf(fmaxf(q + (float)zp, 0.f), 15.f);
+                    wd[i >> 3] |= (uint32_t)u << nibble_shift(i & 7);
+                }
+                out = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+
+            const int64_t j = (c * 32) / G;     // group of this lane
+            if (valid) {
+                qweight[n * KC + c] = out;      // 16 bytes = the 32 codes of this lane
+                if ((lane % LPG) == 0) scales[n * NG + j] = s16;
             }
             if (MODE == W4_ASYM) {
+                // OR the zero-points of 8 consecutive groups (8*LPG lanes) into one word
+                uint32_t z = (valid && (lane % LPG) == 0) ? ((uint32_t)zp << (4 * (int)(j & 7))) : 0u;
 #pragma unroll
-                for (int i = 0; i < ZPB; ++i) {
-                    const int64_t zw = (c0 * 8) / (8 * G) + i;
-                    if (lane == i && zw < ZW) qzeros[n * ZW + zw] = zacc[i];
-                }
+                for (int off = 1; off < 8 * LPG; off <<= 1) z |= __shfl_xor_sync(0xffffffffu, z, off);
+                if (valid && (lane % (8 * LPG)) == 0) qzeros[n * ZW + (j >> 3)] = z;
             }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) cur[i] = nxt[i];
         }
     }
 }
@@ -197,10 +210,10 @@ cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, u
     if (blocks > cap) blocks = cap;
     if (s)
         quant_pack_kernel<G, MODE, true><<<(unsigned)blocks, threads, 0, stream>>>(
-            (const uint4 *)W, N, K, (const float4 *)s, qweight, (unsigned short *)scales, qzeros);
+            (const uint4 *)W, N, K, (const float4 *)s, (uint4 *)qweight, (unsigned short *)scales, qzeros);
     else
         quant_pack_kernel<G, MODE, false><<<(unsigned)blocks, threads, 0, stream>>>(
-            (const uint4 *)W, N, K, nullptr, qweight, (unsigned short *)scales, qzeros);
+            (const uint4 *)W, N, K, nullptr, (uint4 *)qweight, (unsigned short *)scales, qzeros);
     return cudaGetLastError();
 }
 

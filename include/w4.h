@@ -81,7 +81,7 @@ typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
  * w4_quant_pack -- fold, group-quantize and pack a bf16 weight matrix.
  *   (page 5 section 2.2 formulas; page 2 group quantization; page 3 sections
  *    2.2 and 5.3 for the scale shape and the fold)
- *   W        bf16 [N][K], row k-contiguous.
+ *   W        bf16 [N][K], row k-contiguous, 32-byte aligned.
  *   N, K     N >= 1; K >= 8, K % group == 0.
  *   group    32, 64 or 128.
  *   mode     W4_SYM or W4_ASYM.

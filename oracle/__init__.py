@@ -206,6 +206,13 @@ def w4a16_reference(X_bits, qweight, scales, qzeros, K, g, mode, channels=None, 
     return gemm_f64(X_bits, What, threads=threads)
 
 
+def w4a16_abs_reference(X_bits, qweight, scales, qzeros, K, g, mode, threads=1):
+    """sum_k |x[m][k]| * |w^[n][k]| in fp64: the scale of the rounding error of
+    any order of accumulating Y[m][n]."""
+    What = dequant(qweight, scales, qzeros, K, g, mode)
+    return gemm_f64(np.ascontiguousarray(X_bits, dtype=np.uint16) & 0x7FFF, What & 0x7FFF, threads=threads)
+
+
 def e2m1_decode(code: int) -> float:
     """Value of a 4-bit E2M1 code (page 5 section 2.1)."""
     return float(lib().orc_e2m1_decode(int(code)))

@@ -75,6 +75,7 @@ def test_quant_pack_rejects_bad_arguments(w4):
     assert qp(w4, mode=1, z=None) == E           # asymmetric needs qzeros
     assert qp(w4, mode=0, z=FAKE) == E           # symmetric must not get qzeros
     assert qp(w4, W=FAKE + 2) == E               # misaligned bf16 input
+    assert qp(w4, W=FAKE + 16) == E              # W needs 32-byte alignment (256-bit loads)
     assert qp(w4, q=FAKE + 4) == E
     assert qp(w4, s=FAKE + 4) == E
     assert qp(w4, sc=FAKE + 1) == E
