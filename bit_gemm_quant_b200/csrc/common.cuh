@@ -12,6 +12,20 @@ namespace w4 {
 
 constexpr int kNumSMs = 148;             // B200
 
+// Start fetching [p, p + bytes) from HBM into L2 (cp.async.bulk.prefetch); a
+// hint only.  The range is shrunk to its 16-byte-aligned interior so it never
+// leaves the array.
+__device__ __forceinline__ void prefetch_l2(const void *p, size_t bytes)
+{
+    uintptr_t a = ((uintptr_t)p + 15) & ~(uintptr_t)15;
+    const uintptr_t e = ((uintptr_t)p + bytes) & ~(uintptr_t)15;
+    while (a < e) {
+        const uint32_t n = (e - a) > (1u << 20) ? (1u << 20) : (uint32_t)(e - a);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
+        a += n;
+    }
+}
+
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -26,5 +40,7 @@ cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const
                            const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
                            cudaStream_t stream);
 int read_and_clear_device_error();
+// Device address of the library's error word on the current device (nullptr on failure).
+int *device_error_word();
 
 }  // namespace w4

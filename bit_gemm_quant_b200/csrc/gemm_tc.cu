@@ -25,7 +25,7 @@
 // Warp roles (320 threads): warp 0 issues the TMA loads, warp 1 allocates
 // tensor memory and one of its threads issues the MMAs, warps 2..9 dequantize
 // (warp w owns the 32 lanes 32*(w%4).. of tensor memory and every other
-// k-block) and then run the epilogue.  A 4-stage ring couples them with
+// k-block) and then run the epilogue.  A 4- or 6-stage ring couples them with
 // mbarriers: full_b (TMA bytes landed), full_a (4 warps stored their A
 // slice), empty (tcgen05.commit: the MMAs that read the stage are done).
 // Every wait is bounded in time; a wait that runs out records an error code
@@ -46,7 +46,6 @@ static __device__ int g_device_error;
 
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kThreads = 320;
 constexpr int kKB = 64;                      // k per block (one 128-byte swizzle row of bf16)
 constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms; no legitimate wait comes near it
@@ -184,7 +183,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v)
 {
     uint32_t r[8];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -266,9 +281,12 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr)
 
 template <int BN>
 struct TcCfg {
+    static constexpr int kCols = (BN <= 128) ? 256 : 512;               // tensor-memory allocation
+    // pipeline depth: as many 32-column A stages as fit beside the accumulator, at most 6 (even)
+    static constexpr int kStages = ((kCols - BN) / 32 >= 6) ? 6 : 4;
     static constexpr int kACol0 = BN;                                   // A stages follow the BN fp32 accumulator columns
-    static constexpr int kCols = (BN + kStages * 32 <= 256) ? 256 : 512; // tensor-memory allocation
     static constexpr int kStageBytes = BN * 128;                        // activation box bytes
+    static_assert(kACol0 + kStages * 32 <= kCols, "tensor memory overflow");
     static constexpr int kMinBlocks = (BN == 256) ? 1 : 2;
     // kind::f16, fp32 D, bf16 A and B, both K-major, N = BN, M = 128
     static constexpr uint32_t kIdesc =
@@ -289,6 +307,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
                unsigned *__restrict__ counters, int splits, int kb_per_split)
 {
     using C = TcCfg<BN>;
+    constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *sB = smem;                                               // kStages x BN x 128 bytes
@@ -434,12 +453,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
         constexpr int HALF = BN / 2;                  // columns per warp of a lane quarter
         const int cbeg = h * HALF;
         if (have) {
-            for (int c = 0; c < HALF; c += 8) {
-                float acc[8];
-                tmem_ld8(lane_addr + cbeg + c, acc);
+            // columns in chunks of CH (64, or the whole half when it is smaller),
+            // all loads of a chunk issued before one wait
+            constexpr int CH = HALF < 64 ? HALF : 64;
+            for (int c = 0; c < HALF; c += CH) {
+                float acc[CH];
+                if (CH >= 32) {
+#pragma unroll
+                    for (int u = 0; u < CH / 32; ++u) tmem_ld32(lane_addr + cbeg + c + 32 * u, acc + 32 * u);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < CH / 8; ++u) tmem_ld8(lane_addr + cbeg + c + 8 * u, acc + 8 * u);
+                }
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < CH; ++j) {
                     const int m = m0 + cbeg + c + j;
                     if (okn && m < M) {
                         if (splits == 1) Y[(size_t)m * N + n] = __float2bfloat16_rn(acc[j]);
@@ -548,7 +576,7 @@ cudaError_t launch_bn(const CUtensorMap &map, const TcPlan &p, int M, int N, int
                       cudaStream_t stream)
 {
     using C = TcCfg<BN>;
-    size_t smem = 1024 + kStages * C::kStageBytes + 256;
+    size_t smem = 1024 + C::kStages * C::kStageBytes + 256;
     if (C::kMinBlocks == 2 && smem < 80 * 1024) smem = 80 * 1024;   // at most 2 CTAs share an SM's tensor memory
     static bool attr_set = false;
     if (!attr_set) {
@@ -600,6 +628,19 @@ cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const
     case 128: return launch_bn<128>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
     default: return launch_bn<256>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
     }
+}
+
+int *device_error_word()
+{
+    static int *addr[64] = {};                   // per device, resolved once
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = (int *)p;
+    }
+    return addr[dev];
 }
 
 int read_and_clear_device_error()

@@ -11,16 +11,19 @@
 // .../02-core-ideas) section 2.2, x^ = (q - zp) * s, rounded once to bf16.
 //
 // Design (HBM-bound: 0.5 B of codes + 1/64 B of scale per weight at g = 128):
-//   * a tile is 16 output channels and all of K; a CTA loops over the tiles
-//     blockIdx.x, blockIdx.x + gridDim.x, ... (two CTAs per SM, every CTA the
-//     same number of tiles); its 8 warps split K into 512-wide super-chunks
-//     (warp w takes super-chunks w, w+8, ...) and sum their partial tiles in
-//     double-buffered shared memory after the last super-chunk of each tile
-//     (no global scratch); each warp loads its next work item before it
-//     computes the current one;
+//   * a CTA (4 warps) owns a tile of 16 output channels and all of K; its
+//     warps split K into 512-wide super-chunks (warp w takes super-chunks w,
+//     w+4, ...) and sum their partial tiles in shared memory at the end (no
+//     global scratch); small CTAs keep many tiles resident per SM;
+//   * at launch the CTA's first threads ask L2 to fetch the tile's codes,
+//     scales and zero-points (cp.async.bulk.prefetch, one instruction per
+//     channel), so every byte of the tile is requested from HBM at once and
+//     the warps' own loads see L2 latency; small CTAs keep several tiles per
+//     SM in flight;
 //   * lane (g, t) = (lane/4, lane%4) of a warp loads, for channels g and g+8,
-//     the 64 contiguous bytes (128 codes) at k = 512*sc + 128*t: all of its
-//     loads are issued before any arithmetic (8 x 16 B per lane);
+//     the 64 contiguous bytes (128 codes) at k = 512*sc + 128*t, with the
+//     scales and zero-points of their groups, and the activations one 32-wide
+//     step ahead;
 //   * each 32-bit word of codes gives four bf16x2 pairs of ADJACENT elements
 //     with one shift and one LOP3 (the packed layout keeps even elements in
 //     the low half-word), as 128 + u via the bf16 exponent of 128;
@@ -40,15 +43,6 @@
 
 namespace w4 {
 namespace {
-
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
 
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
 {
@@ -108,77 +102,85 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupC
     return bf2_fma(D, gc.shi, bf2_mul(D, gc.slo));
 }
 
-constexpr int kWarps = 8;
-
-// A warp's work item is one 512-wide super-chunk of K for the 16 channels of
-// a tile: 4 x 16 bytes of codes per lane for each of its two channels.
-struct Item {
-    uint4 a[4], b[4];
-};
+constexpr int kWarps = 4;
 
 template <int G, int MODE>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+__global__ void __launch_bounds__(kWarps * 32)
 gemv_kernel(const uint4 *__restrict__ X, int M, int N, int K, const uint4 *__restrict__ qweight,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
             __nv_bfloat16 *__restrict__ Y)
 {
     constexpr int QPG = G / 32;                  // 16-byte code chunks per group
-    __shared__ float red[2][kWarps][32][4];
+    constexpr int NGI = 4 / QPG;                 // groups per super-chunk and channel, per lane
+    __shared__ float red[kWarps][32][4];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int KQ = K >> 5;                       // 16-byte code chunks per channel
     const int NG = K / G, ZW = (NG + 7) >> 3;
-    const int ntiles = (N + 15) >> 4;
-    const int nsc = (KQ + 15) >> 4;              // 512-wide super-chunks per channel
-    const int per_warp = (nsc + kWarps - 1) / kWarps;
-    const int my_tiles = (ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    const int items = my_tiles * per_warp;
+    const int r0 = (int)blockIdx.x * 16;
+    const int rA = r0 + g, rB = rA + 8;
+    const bool okA = rA < N, okB = rB < N;
+    const int rows = min(16, N - r0);
+
+    // the whole tile, HBM -> L2, before any thread waits on a load
+    if (threadIdx.x < rows) prefetch_l2(qweight + (size_t)(r0 + threadIdx.x) * KQ, (size_t)KQ * 16);
+    else if (threadIdx.x == 16) prefetch_l2(scales + (size_t)r0 * NG, (size_t)rows * NG * 2);
+    else if (threadIdx.x == 17 && MODE == W4_ASYM) prefetch_l2(qzeros + (size_t)r0 * ZW, (size_t)rows * ZW * 4);
+
     const bool has_x = g < M;
     const uint4 *xrow = X + (size_t)(has_x ? g : 0) * (K >> 3);
+    const uint4 *qa = qweight + (size_t)(okA ? rA : 0) * KQ;
+    const uint4 *qb = qweight + (size_t)(okB ? rB : 0) * KQ;
+    const unsigned short *sa_row = scales + (size_t)(okA ? rA : 0) * NG;
+    const unsigned short *sb_row = scales + (size_t)(okB ? rB : 0) * NG;
+    const uint32_t *za_row = qzeros + (size_t)(okA ? rA : 0) * ZW;
+    const uint32_t *zb_row = qzeros + (size_t)(okB ? rB : 0) * ZW;
 
-    auto fetch = [&](int it, Item &d) {
-        const int tile = (int)blockIdx.x + (it / per_warp) * (int)gridDim.x;
-        const int q0 = (warp + kWarps * (it % per_warp)) * 16 + t * 4;
-        const int rA = tile * 16 + g, rB = rA + 8;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // warp w takes the 512-wide super-chunks w, w+4, ...; lane t their chunks 4t..4t+3
+    for (int s0 = warp * 16; s0 < KQ; s0 += kWarps * 16) {
+        const int q0 = s0 + 4 * t;
+        uint4 a[4], b[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const bool ok = q0 + i < KQ;
-            d.a[i] = (ok && rA < N) ? ld_stream(qweight + (size_t)rA * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
-            d.b[i] = (ok && rB < N) ? ld_stream(qweight + (size_t)rB * KQ + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+            a[i] = (ok && okA) ? __ldg(qa + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+            b[i] = (ok && okB) ? __ldg(qb + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
         }
-    };
-
-    Item cur, nxt;
-    if (items > 0) fetch(0, cur);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int it = 0; it < items; ++it) {
-        if (it + 1 < items) fetch(it + 1, nxt);
-        const int tile = (int)blockIdx.x + (it / per_warp) * (int)gridDim.x;
-        const int q0 = (warp + kWarps * (it % per_warp)) * 16 + t * 4;
-        const int rA = tile * 16 + g, rB = rA + 8;
-        const bool okA = rA < N, okB = rB < N;
+        unsigned short sa[NGI], sb[NGI];
+        uint32_t za[NGI], zb[NGI];
+#pragma unroll
+        for (int u = 0; u < NGI; ++u) {
+            const int qi = q0 + u * QPG;
+            const bool ok = qi < KQ;
+            const int j = ok ? (qi * 32) / G : 0;
+            sa[u] = (ok && okA) ? __ldg(sa_row + j) : (unsigned short)0;
+            sb[u] = (ok && okB) ? __ldg(sb_row + j) : (unsigned short)0;
+            if (MODE == W4_ASYM) {
+                za[u] = (ok && okA) ? (__ldg(za_row + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
+                zb[u] = (ok && okB) ? (__ldg(zb_row + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
+            } else {
+                za[u] = zb[u] = 8u;
+            }
+        }
+        uint4 xv[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) xv[w] = (has_x && q0 < KQ) ? __ldg(xrow + q0 * 4 + w) : make_uint4(0u, 0u, 0u, 0u);
         GroupConst ca, cb;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int qi = q0 + i;
-            const bool ok = qi < KQ;
-            if (i % QPG == 0) {
-                const int j = ok ? (qi * 32) / G : 0;
-                uint32_t za = 8u, zb = 8u;
-                if (MODE == W4_ASYM) {
-                    za = okA ? (__ldg(qzeros + (size_t)rA * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
-                    zb = okB ? (__ldg(qzeros + (size_t)rB * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
-                }
-                ca = group_const(okA ? __ldg(scales + (size_t)rA * NG + j) : (unsigned short)0, (int)za);
-                cb = group_const(okB ? __ldg(scales + (size_t)rB * NG + j) : (unsigned short)0, (int)zb);
-            }
-            uint4 xv[4];
+            uint4 xn[4];                         // activations of the next 32-wide step
+            const bool okn = has_x && i < 3 && qi + 1 < KQ;
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-                xv[w] = (has_x && ok) ? __ldg(xrow + qi * 4 + w) : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t wa[4] = {cur.a[i].x, cur.a[i].y, cur.a[i].z, cur.a[i].w};
-            const uint32_t wb[4] = {cur.b[i].x, cur.b[i].y, cur.b[i].z, cur.b[i].w};
+            for (int w = 0; w < 4; ++w) xn[w] = okn ? __ldg(xrow + (qi + 1) * 4 + w) : make_uint4(0u, 0u, 0u, 0u);
+            if (i % QPG == 0) {
+                ca = group_const(sa[i / QPG], (int)za[i / QPG]);
+                cb = group_const(sb[i / QPG], (int)zb[i / QPG]);
+            }
+            const uint32_t wa[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+            const uint32_t wb[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const uint32_t a0 = dequant_pair(wa[w], 0, ca), a1 = dequant_pair(wa[w], 1, ca);
@@ -188,29 +190,25 @@ gemv_kernel(const uint4 *__restrict__ X, int M, int N, int K, const uint4 *__res
                 mma_bf16_16816(acc, a0, b0, a1, b1, xv[w].x, xv[w].y);
                 mma_bf16_16816(acc, a2, b2, a3, b3, xv[w].z, xv[w].w);
             }
+#pragma unroll
+            for (int w = 0; w < 4; ++w) xv[w] = xn[w];
         }
-        if (it % per_warp == per_warp - 1) {     // last super-chunk of this tile: reduce the 8 warps
-            const int buf = (it / per_warp) & 1;
+    }
+
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                red[buf][warp][lane][i] = acc[i];
-                acc[i] = 0.f;
-            }
-            __syncthreads();
-            if (warp == 0) {
-                float sm[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < 4; ++i) red[warp][lane][i] = acc[i];
+    __syncthreads();
+    if (warp == 0) {
+        float sm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int w = 0; w < kWarps; ++w)
+        for (int w = 0; w < kWarps; ++w)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) sm[i] += red[buf][w][lane][i];
-                const int m0 = 2 * t, m1 = 2 * t + 1;   // tokens of c0/c2 and c1/c3
-                if (okA && m0 < M) Y[(size_t)m0 * N + rA] = __float2bfloat16_rn(sm[0]);
-                if (okA && m1 < M) Y[(size_t)m1 * N + rA] = __float2bfloat16_rn(sm[1]);
-                if (okB && m0 < M) Y[(size_t)m0 * N + rB] = __float2bfloat16_rn(sm[2]);
-                if (okB && m1 < M) Y[(size_t)m1 * N + rB] = __float2bfloat16_rn(sm[3]);
-            }
-        }
-        cur = nxt;
+            for (int i = 0; i < 4; ++i) sm[i] += red[w][lane][i];
+        const int m0 = 2 * t, m1 = 2 * t + 1;    // tokens of c0/c2 and c1/c3
+        if (okA && m0 < M) Y[(size_t)m0 * N + rA] = __float2bfloat16_rn(sm[0]);
+        if (okA && m1 < M) Y[(size_t)m1 * N + rA] = __float2bfloat16_rn(sm[1]);
+        if (okB && m0 < M) Y[(size_t)m0 * N + rB] = __float2bfloat16_rn(sm[2]);
+        if (okB && m1 < M) Y[(size_t)m1 * N + rB] = __float2bfloat16_rn(sm[3]);
     }
 }
 
@@ -218,11 +216,7 @@ template <int G, int MODE>
 cudaError_t launch_g_mode(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                           const void *scales, const uint32_t *qzeros, void *Y, cudaStream_t stream)
 {
-    // as many CTAs as two per SM allow, rounded so that every CTA gets the same number of tiles
-    const int64_t ntiles = (N + 15) / 16;
-    const int64_t slots = (int64_t)kNumSMs * 2;
-    const int64_t per_cta = (ntiles + slots - 1) / slots;
-    const int64_t blocks = (ntiles + per_cta - 1) / per_cta;
+    const int64_t blocks = (N + 15) / 16;       // one 16-channel tile per CTA
     gemv_kernel<G, MODE><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
         (const uint4 *)X, (int)M, (int)N, (int)K, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
         (__nv_bfloat16 *)Y);

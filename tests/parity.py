@@ -53,7 +53,8 @@ def assert_y_elementwise(Y: np.ndarray, Y_ref: np.ndarray, Y_abs: np.ndarray, K:
     rounding of an fp32 sum whose accumulation error is at most e."""
     e = K * 2.0 ** -22 * Y_abs
     bound = 2.0 ** -8 * (np.abs(Y_ref) + e) + e
-    bad = np.abs(Y - Y_ref) > bound
+    bad = ~(np.abs(Y - Y_ref) <= bound)          # NaN or Inf counts as outside
+    assert np.isfinite(Y).all(), "%s: non-finite outputs" % what
     assert not bad.any(), "%s: %d outputs outside the rounding bound, first %s: got %r, ref %r, bound %r" % (
         what, int(bad.sum()), tuple(np.argwhere(bad)[0]), Y[bad][0], Y_ref[bad][0], bound[bad][0])
 

@@ -385,3 +385,32 @@ def test_e2m1_value_set(oracle_mod):
     vals = {oracle_mod.e2m1_decode(c) for c in range(16)}
     assert vals == set(fx["values"]) | {-0.0}
     assert sorted(vals) == sorted(set(fx["values"]))
+
+
+# ------------------------------------------------- rounding of quotients ---
+
+def test_rint_of_fp32_quotient_equals_exact_rounding():
+    """For fp32 x and an fp16-representable d > 0, rint(fl32(x/d)) equals the
+    round-half-even of the exact quotient: the IEEE codes of page 5 section 2.2
+    are the nearest codes in exact arithmetic.  Checked on a million quotients
+    concentrated at and next to half-integers (exact comparison in fp64: b*d and
+    x are exact there and the sign of x - b*d is exact)."""
+    rng = np.random.default_rng(13)
+    n = 1_000_000
+    d = rng.integers(0x0001, 0x7BFF, n).astype(np.uint16).view(np.float16).astype(np.float32)
+    b = rng.integers(-16, 16, n).astype(np.float64) + 0.5
+    bd = (b * d.astype(np.float64)).astype(np.float32)            # exact: b*d has <= 16 bits
+    ulps = rng.integers(-4, 5, n).astype(np.int32)
+    x = (bd.view(np.int32) + ulps).view(np.float32)              # ties and their neighbours
+    x[::7] = (rng.standard_normal(n // 7 + 1)[: x[::7].size] * 8 * d[::7]).astype(np.float32)
+    ok = np.isfinite(x) & (d > 0)
+    x, d = x[ok], d[ok]
+    q32 = np.rint(x / d)                                          # numpy float32 division is IEEE
+    X, D = x.astype(np.float64), d.astype(np.float64)
+    f = np.floor(X / D)
+    for _ in range(2):                                            # make f = floor(x/d) exactly
+        f = np.where(X < f * D, f - 1, f)
+        f = np.where(X >= (f + 1) * D, f + 1, f)
+    h = (f + 0.5) * D                                             # exact in fp64
+    exact = np.where(X > h, f + 1, np.where(X < h, f, np.where(f % 2 == 0, f, f + 1)))
+    assert np.array_equal(q32.astype(np.float64), exact)
