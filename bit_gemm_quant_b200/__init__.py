@@ -40,6 +40,8 @@ def lib() -> ctypes.CDLL:
         L.w4a16_workspace_bytes.restype = SZ
         L.w4a16_gemm.argtypes = [P, I64, I64, I64, P, P, P, I, I, P, P, SZ, P]
         L.w4a16_gemm.restype = I
+        L.w4a16_gemm_noalloc.argtypes = [P, I64, I64, I64, P, P, P, I, I, P, P]
+        L.w4a16_gemm_noalloc.restype = I
         L.w4_status_string.argtypes = [I]
         L.w4_status_string.restype = ctypes.c_char_p
         L.w4_layout_version.argtypes = []
@@ -63,6 +65,10 @@ def w4a16_workspace_bytes(M, N, K, group) -> int:
 def w4a16_gemm(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace, workspace_bytes, stream) -> int:
     return lib().w4a16_gemm(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace,
                             workspace_bytes, stream)
+
+
+def w4a16_gemm_noalloc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, stream) -> int:
+    return lib().w4a16_gemm_noalloc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, stream)
 
 
 def w4_status_string(status: int) -> str:
@@ -132,4 +138,21 @@ def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None
                     _ptr(workspace), wbytes, _stream_handle(stream))
     if st != W4_OK:
         raise W4Error(st, "w4a16_gemm")
+    return Y
+
+
+def gemm_noalloc(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None, out=None, stream=None):
+    """Like ``gemm`` for callers that cannot allocate device scratch: the
+    split-K scratch is the library's own fixed array (shapes that need more
+    than it holds raise W4Error with W4_ERR_UNSUPPORTED).  Only the output is
+    allocated here, and only when ``out`` is None."""
+    import torch
+    M, K = X.shape
+    if N is None:
+        N = qweight.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    st = w4a16_gemm_noalloc(_ptr(X), M, N, K, _ptr(qweight), _ptr(scales), _ptr(qzeros), group, mode, _ptr(Y),
+                            _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4a16_gemm_noalloc")
     return Y

@@ -36,6 +36,8 @@ cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const ui
                         const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                         cudaStream_t stream);
 size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
+// byte range of the split-K tile counters inside that workspace (0 bytes if none)
+void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size_t *bytes);
 cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                            const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
                            cudaStream_t stream);

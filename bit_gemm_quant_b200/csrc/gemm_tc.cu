@@ -603,6 +603,18 @@ cudaError_t launch_bn(const CUtensorMap &map, const TcPlan &p, int M, int N, int
 
 size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K) { return plan_tc(M, N, K).ws_bytes; }
 
+void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size_t *bytes)
+{
+    const TcPlan p = plan_tc(M, N, K);
+    *offset = 0;
+    *bytes = 0;
+    if (p.splits > 1) {
+        const size_t part = (size_t)p.splits * M * N * sizeof(float);
+        *offset = (part + 255) & ~(size_t)255;
+        *bytes = p.ws_bytes - *offset;
+    }
+}
+
 cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                            const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
                            cudaStream_t stream)

@@ -125,6 +125,32 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
                      const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                      void *workspace, size_t workspace_bytes, w4_stream_t stream);
 
+/*
+ * w4a16_gemm_noalloc -- w4a16_gemm for callers that cannot allocate device
+ * memory (a stream capture that must not allocate, a host whose allocator
+ * owns all device memory, a plug-in that only receives its input and output
+ * buffers).  The pages have no counterpart to this entry point: it only
+ * changes where the split-K scratch lives.
+ *   Arguments, results and errors are those of w4a16_gemm without the
+ *   workspace.  The split-K scratch is a library-owned device array of
+ *   W4_NOALLOC_SCRATCH_BYTES bytes that every GPU which loads the library
+ *   holds until the process exits; shapes whose w4a16_workspace_bytes
+ *   exceeds it are rejected with W4_ERR_UNSUPPORTED before anything is
+ *   launched.  No device memory is allocated or freed.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture on the device.
+ *   Each call first clears the array's split-K counters with
+ *   cudaMemsetAsync on `stream`.  All calls share the array: calls ordered
+ *   on one stream are safe, calls whose work overlaps on the GPU (unordered
+ *   streams, several host threads) race and give wrong results.
+ */
+#define W4_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
+                             const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
+                             w4_stream_t stream);
+
 /* Text for a status code; never NULL. */
 const char *w4_status_string(int status);
 
