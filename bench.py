@@ -108,7 +108,7 @@ def problems_for(workload: str):
 
 
 def kernel_name(M: int) -> str:
-    return "w4a16_gemv" if M <= 8 else "w4a16_gemm_tc"
+    return "w4a16_gemv" if M <= 16 else "w4a16_gemm_tc"
 
 
 class Launch:

@@ -11,6 +11,9 @@ bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
 
 bool mode_ok(int m) { return m == W4_SYM || m == W4_ASYM; }
 
+// batches up to this size run the GEMV (two MMA token groups of 8)
+constexpr int64_t kGemvMaxM = 16;
+
 // int64 products used for sizes must not overflow
 bool fits(int64_t a, int64_t b) { return a > 0 && b > 0 && a <= INT64_MAX / b; }
 
@@ -49,7 +52,7 @@ w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group)
 {
     (void)group;
-    if (M <= 8 || M < 1 || N < 1 || K < 1) return 0;
+    if (M <= kGemvMaxM || M < 1 || N < 1 || K < 1) return 0;
     return w4::tc_workspace_bytes(M, N, K);
 }
 
@@ -69,8 +72,8 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
     if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256))))
         return W4_ERR_INVALID_ARG;
     cudaError_t e;
-    if (M <= 8) {
-        if (N > INT32_MAX - 16 || K > INT32_MAX) return W4_ERR_UNSUPPORTED;
+    if (M <= kGemvMaxM) {
+        if (N > INT32_MAX - 16 || K > INT32_MAX || M * K > INT32_MAX) return W4_ERR_UNSUPPORTED;
         e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, Y, (cudaStream_t)stream);
     } else {
         // tensor-core path: 32-bit indices, TMA extents

@@ -1,4 +1,4 @@
-// w4a16_gemm, M > 8: the tensor-core path (tcgen05, tensor memory, TMA).
+// w4a16_gemm, M > 16: the tensor-core path (tcgen05, tensor memory, TMA).
 //
 // Method: page 4 (llm-glossary.tokens-kit.com/terms/quantization-methods/, GPTQ
 // section) notes that large prefill GEMMs are governed by the dequantize /

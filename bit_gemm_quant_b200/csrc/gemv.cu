@@ -1,29 +1,34 @@
-// w4a16_gemm, M <= 8: the decode GEMV / skinny path.
+// w4a16_gemm, M <= 16: the decode GEMV / skinny path.
 //
 // Method: page 2 (learn.longtimenohack.com .../quantization.html) opens with
 // "reading weights is the top cost of decode", page 4
 // (llm-glossary.tokens-kit.com/terms/quantization-methods/, GPTQ section) with
 // "small-batch decode profits from the weight bandwidth", and page 3
 // (blog.freezetheflame.cc quantization deep dive) section 1.2 with "fuse
-// dequantize into the GEMM so the weights stay 4-bit in HBM"; section 3.1 of
-// the same page sketches Marlin, which unpacks INT4 in registers and feeds
-// mma.sync.  Dequantization follows page 5 (ai-infra.cypggs.com
-// .../02-core-ideas) section 2.2, x^ = (q - zp) * s, rounded once to bf16.
+// dequantize into the GEMM so the weights stay 4-bit in HBM"; section 2.2 of
+// the same page prefetches the group scales to shared memory, and its section
+// 3.1 sketches Marlin, which unpacks INT4 in registers and feeds mma.sync.
+// Dequantization follows page 5 (ai-infra.cypggs.com .../02-core-ideas)
+// section 2.2, x^ = (q - zp) * s, rounded once to bf16.
 //
-// Design (HBM-bound: 0.5 B of codes + 1/64 B of scale per weight at g = 128):
-//   * a CTA (4 warps) owns a tile of 16 output channels and all of K; its
-//     warps split K into 512-wide super-chunks (warp w takes super-chunks w,
-//     w+4, ...) and sum their partial tiles in shared memory at the end (no
-//     global scratch); small CTAs keep many tiles resident per SM;
-//   * at launch the CTA's first threads ask L2 to fetch the tile's codes,
-//     scales and zero-points (cp.async.bulk.prefetch, one instruction per
-//     channel), so every byte of the tile is requested from HBM at once and
-//     the warps' own loads see L2 latency; small CTAs keep several tiles per
-//     SM in flight;
-//   * lane (g, t) = (lane/4, lane%4) of a warp loads, for channels g and g+8,
-//     the 64 contiguous bytes (128 codes) at k = 512*sc + 128*t, with the
-//     scales and zero-points of their groups, and the activations one 32-wide
-//     step ahead;
+// Design (HBM-bound: 0.5 B of codes + 1/64 B of scale per weight at g = 128;
+// the dequantization costs about 2.5 issue slots per weight, which is close to
+// the issue budget of the SMs at HBM speed, so the kernel must stream the codes
+// without spending instructions on it):
+//   * a CTA (4 warps) owns a tile of 16 output channels and all of K; warp w
+//     takes the 256-wide k-boxes w, w+4, w+8, ... and the four partial tiles
+//     are summed in shared memory at the end (no global scratch);
+//   * the codes stream HBM -> shared memory by TMA (one 2-D box of 16 rows x
+//     128 bytes per k-box, 128-byte swizzle), three boxes in flight per warp on
+//     the warp's own mbarrier ring, so a resident CTA keeps 24 KB of reads
+//     outstanding and the loads cost the warps one instruction per box;
+//   * per k-box, each lane turns one (channel, group) scale and zero-point into
+//     the bf16x2 constants below and parks them in the warp's shared-memory
+//     slot, where the lanes that need them read them back (the scales and
+//     zero-points of the next box are loaded while this one is computed);
+//   * lane (g, t) = (lane/4, lane%4) reads, for channels g and g+8, the 16-byte
+//     chunks t and t+4 of the box (the swizzle makes these reads free of bank
+//     conflicts) and the activations of the same k from global memory;
 //   * each 32-bit word of codes gives four bf16x2 pairs of ADJACENT elements
 //     with one shift and one LOP3 (the packed layout keeps even elements in
 //     the low half-word), as 128 + u via the bf16 exponent of 128;
@@ -35,14 +40,59 @@
 //   * mma.sync m16n8k16 (bf16 in, fp32 accumulate) takes those registers as
 //     its A fragment directly: the k-order inside an MMA is free, so a
 //     thread's logical columns (2t, 2t+1) and (2t+8, 2t+9) are mapped to the
-//     physical elements 8w+4h+{0,1} and 8w+4h+{2,3} of its own words, and the
-//     activation fragment for token g is then the plain 16-byte chunk
-//     X[g][k + 8w .. k + 8w + 7];
-//   * tokens occupy the MMA's N = 8 columns; lanes with g >= M feed zeros.
+//     physical elements {0,1} and {2,3} (then {4,5} and {6,7}) of its own
+//     words, and the activation fragment for token g is then the plain 16-byte
+//     chunk of X[g] at the word's k;
+//   * tokens occupy the MMA's N = 8 columns, MT groups of 8 tokens (M <= 8 * MT);
+//     lanes whose token is >= M feed zeros.
+// Every wait on an mbarrier is bounded in time; a wait that runs out records
+// an error code (read by w4_device_error), and the warp stops computing, waits
+// (again bounded) for its own copies in flight and returns.
 #include "common.cuh"
+
+#include <cuda.h>
 
 namespace w4 {
 namespace {
+
+constexpr int kWarps = 4;
+constexpr int kStages = 3;                       // k-boxes in flight per warp
+constexpr int kBoxK = 256;                       // k per box: 32 words of 8 codes
+constexpr int kBoxBytes = 16 * 128;              // 16 channels x 128 bytes
+constexpr uint64_t kWaitLimitNs = 200000000ull;  // 200 ms; a box lands in microseconds
+constexpr int kErrGemvWait = 0x201, kErrGemvDrain = 0x202;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity; false after kWaitLimitNs.
+__device__ __noinline__ bool wait_box(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kWaitLimitNs) return false;
+    return true;
+}
 
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
 {
@@ -77,150 +127,224 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 
 // Per-(channel, group) dequantization constants, each duplicated into both
 // halves of a bf16x2: s_hi = bf16_rne(s16), s_lo = s16 - s_hi, Z = 128 + zp.
-struct GroupConst {
-    uint32_t shi, slo, z;
-};
-
-__device__ __forceinline__ GroupConst group_const(unsigned short s16bits, int zp)
+__device__ __forceinline__ uint4 group_const(unsigned short s16bits, uint32_t zp)
 {
     const float sf = __half2float(__ushort_as_half(s16bits));
     const __nv_bfloat16 hi = __float2bfloat16_rn(sf);
     const __nv_bfloat16 lo = __float2bfloat16_rn(sf - __bfloat162float(hi));   // exact
     const uint32_t h = __bfloat16_as_ushort(hi), l = __bfloat16_as_ushort(lo);
-    GroupConst gc;
-    gc.shi = h | (h << 16);
-    gc.slo = l | (l << 16);
-    gc.z = 0x43004300u | ((uint32_t)zp << 16) | (uint32_t)zp;
-    return gc;
+    return make_uint4(h | (h << 16), l | (l << 16), 0x43004300u | (zp << 16) | zp, 0u);
 }
 
-// w^ for elements (8c+2j, 8c+2j+1) of packed word q.
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupConst &gc)
+// w^ for elements (2j, 2j+1) of packed word q.
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const uint4 &gc)
 {
     const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) | 0x43004300u;   // 128 + u, as bf16x2
     const uint32_t D = bf2_sub(v, gc.z);
-    return bf2_fma(D, gc.shi, bf2_mul(D, gc.slo));
+    return bf2_fma(D, gc.x, bf2_mul(D, gc.y));
 }
 
-constexpr int kWarps = 4;
-
-template <int G, int MODE>
-__global__ void __launch_bounds__(kWarps * 32)
-gemv_kernel(const uint4 *__restrict__ X, int M, int N, int K, const uint4 *__restrict__ qweight,
-            const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
-            __nv_bfloat16 *__restrict__ Y)
+__device__ __forceinline__ uint4 ldg_x(const uint4 *p, bool ok)
 {
-    constexpr int QPG = G / 32;                  // 16-byte code chunks per group
-    constexpr int NGI = 4 / QPG;                 // groups per super-chunk and channel, per lane
-    __shared__ float red[kWarps][32][4];
+    return ok ? __ldg(p) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <int G, int MODE, int MT>
+__global__ void __launch_bounds__(kWarps * 32, 6)
+gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict__ X, int M, int N, int K,
+            const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
+            __nv_bfloat16 *__restrict__ Y, int *err)
+{
+    constexpr int GPB = kBoxK / G;               // groups per box and channel
+    constexpr int CPL = 16 * GPB / 32;           // constants computed per lane and box
+    __shared__ __align__(1024) uint8_t sbox[kWarps][kStages][kBoxBytes];
+    __shared__ uint4 sconst[kWarps][16 * GPB];
+    __shared__ float red[kWarps][32][4 * MT];
+    __shared__ __align__(8) uint64_t full[kWarps][kStages];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int KQ = K >> 5;                       // 16-byte code chunks per channel
     const int NG = K / G, ZW = (NG + 7) >> 3;
+    const int NB = (K + kBoxK - 1) / kBoxK;      // k-boxes per channel
+    const int nbw = (NB - warp + kWarps - 1) / kWarps;   // boxes of this warp: warp, warp+4, ...
     const int r0 = (int)blockIdx.x * 16;
-    const int rA = r0 + g, rB = rA + 8;
-    const bool okA = rA < N, okB = rB < N;
-    const int rows = min(16, N - r0);
 
-    // the whole tile, HBM -> L2, before any thread waits on a load
-    if (threadIdx.x < rows) prefetch_l2(qweight + (size_t)(r0 + threadIdx.x) * KQ, (size_t)KQ * 16);
-    else if (threadIdx.x == 16) prefetch_l2(scales + (size_t)r0 * NG, (size_t)rows * NG * 2);
-    else if (threadIdx.x == 17 && MODE == W4_ASYM) prefetch_l2(qzeros + (size_t)r0 * ZW, (size_t)rows * ZW * 4);
+    const uint32_t bar0 = smem_u32(&full[warp][0]);
+    const uint32_t box0 = smem_u32(&sbox[warp][0][0]);
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8 * s));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_q) : "memory");
+    }
+    __syncwarp();
+    auto issue = [&](int i) {                    // lane 0: box i of this warp into stage i % kStages
+        const int s = i % kStages;
+        const int b = warp + kWarps * i;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar0 + 8 * s),
+                     "r"(kBoxBytes)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+            "[%2];" ::"r"(box0 + s * kBoxBytes),
+            "l"(&tmap_q), "r"(bar0 + 8 * s), "r"(b * 32), "r"(r0)
+            : "memory");
+    };
+    if (lane == 0)
+        for (int i = 0; i < kStages && i < nbw; ++i) issue(i);
 
-    const bool has_x = g < M;
-    const uint4 *xrow = X + (size_t)(has_x ? g : 0) * (K >> 3);
-    const uint4 *qa = qweight + (size_t)(okA ? rA : 0) * KQ;
-    const uint4 *qb = qweight + (size_t)(okB ? rB : 0) * KQ;
-    const unsigned short *sa_row = scales + (size_t)(okA ? rA : 0) * NG;
-    const unsigned short *sb_row = scales + (size_t)(okB ? rB : 0) * NG;
-    const uint32_t *za_row = qzeros + (size_t)(okA ? rA : 0) * ZW;
-    const uint32_t *zb_row = qzeros + (size_t)(okB ? rB : 0) * ZW;
-
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    // warp w takes the 512-wide super-chunks w, w+4, ...; lane t their chunks 4t..4t+3
-    for (int s0 = warp * 16; s0 < KQ; s0 += kWarps * 16) {
-        const int q0 = s0 + 4 * t;
-        uint4 a[4], b[4];
+    // scales / zero-points of the constants this lane computes for box i
+    unsigned short sv[CPL];
+    uint32_t zv[CPL];
+    auto load_consts = [&](int i) {
+        const int b = warp + kWarps * i;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool ok = q0 + i < KQ;
-            a[i] = (ok && okA) ? __ldg(qa + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
-            b[i] = (ok && okB) ? __ldg(qb + q0 + i) : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < CPL; ++u) {
+            const int idx = lane + 32 * u, row = r0 + (idx & 15), j = b * GPB + (idx >> 4);
+            const bool ok = row < N && j < NG;
+            sv[u] = ok ? __ldg(scales + (size_t)row * NG + j) : (unsigned short)0;
+            if (MODE == W4_ASYM) zv[u] = ok ? (__ldg(qzeros + (size_t)row * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
+            else zv[u] = 8u;
         }
-        unsigned short sa[NGI], sb[NGI];
-        uint32_t za[NGI], zb[NGI];
+    };
+    if (nbw > 0) load_consts(0);
+
+    float acc[MT][4];
 #pragma unroll
-        for (int u = 0; u < NGI; ++u) {
-            const int qi = q0 + u * QPG;
-            const bool ok = qi < KQ;
-            const int j = ok ? (qi * 32) / G : 0;
-            sa[u] = (ok && okA) ? __ldg(sa_row + j) : (unsigned short)0;
-            sb[u] = (ok && okB) ? __ldg(sb_row + j) : (unsigned short)0;
-            if (MODE == W4_ASYM) {
-                za[u] = (ok && okA) ? (__ldg(za_row + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
-                zb[u] = (ok && okB) ? (__ldg(zb_row + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
-            } else {
-                za[u] = zb[u] = 8u;
-            }
+    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+
+    bool ok = true;
+    int i = 0;
+    for (; i < nbw; ++i) {
+        const int b = warp + kWarps * i;
+        const int s = i % kStages;
+        // constants of this box into the warp's slot, then the next box's loads
+        __syncwarp();                            // every lane is done with the previous box's slot
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) sconst[warp][lane + 32 * u] = group_const(sv[u], zv[u]);
+        if (i + 1 < nbw) load_consts(i + 1);
+        __syncwarp();
+        if (!wait_box(bar0 + 8 * s, (uint32_t)(i / kStages) & 1u)) {
+            ok = false;
+            break;
         }
-        uint4 xv[4];
+        // this lane's codes: channels g and g+8, chunks t and t+4 (128-byte swizzle)
+        const uint8_t *bx = &sbox[warp][s][0];
+        const uint4 qa0 = *(const uint4 *)(bx + g * 128 + ((t ^ g) << 4));
+        const uint4 qa1 = *(const uint4 *)(bx + g * 128 + (((t + 4) ^ g) << 4));
+        const uint4 qb0 = *(const uint4 *)(bx + (g + 8) * 128 + ((t ^ g) << 4));
+        const uint4 qb1 = *(const uint4 *)(bx + (g + 8) * 128 + (((t + 4) ^ g) << 4));
+        __syncwarp();                            // the stage is read: refill it
+        if (lane == 0 && i + kStages < nbw) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(i + kStages);
+        }
 #pragma unroll
-        for (int w = 0; w < 4; ++w) xv[w] = (has_x && q0 < KQ) ? __ldg(xrow + q0 * 4 + w) : make_uint4(0u, 0u, 0u, 0u);
-        GroupConst ca, cb;
+        for (int h = 0; h < 2; ++h) {
+            const int c = t + 4 * h;             // chunk of this half
+            const int k0 = b * kBoxK + c * 32;   // first k of the chunk
+            const bool kin = k0 < K;             // K is a multiple of 32: chunks are whole
+            const uint4 ca = sconst[warp][(g) + 16 * ((c * 32) / G)];
+            const uint4 cb = sconst[warp][(g + 8) + 16 * ((c * 32) / G)];
+            const uint4 wa4 = h ? qa1 : qa0, wb4 = h ? qb1 : qb0;
+            const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
+            const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
+            uint4 xv[MT][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int qi = q0 + i;
-            uint4 xn[4];                         // activations of the next 32-wide step
-            const bool okn = has_x && i < 3 && qi + 1 < KQ;
+            for (int mt = 0; mt < MT; ++mt) {
+                const int tok = g + 8 * mt;
+                const uint4 *xrow = X + ((size_t)(tok < M ? tok : 0) * K + k0) / 8;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) xn[w] = okn ? __ldg(xrow + (qi + 1) * 4 + w) : make_uint4(0u, 0u, 0u, 0u);
-            if (i % QPG == 0) {
-                ca = group_const(sa[i / QPG], (int)za[i / QPG]);
-                cb = group_const(sb[i / QPG], (int)zb[i / QPG]);
+                for (int w = 0; w < 4; ++w) xv[mt][w] = ldg_x(xrow + w, kin && tok < M);
             }
-            const uint32_t wa[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
-            const uint32_t wb[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const uint32_t a0 = dequant_pair(wa[w], 0, ca), a1 = dequant_pair(wa[w], 1, ca);
                 const uint32_t a2 = dequant_pair(wa[w], 2, ca), a3 = dequant_pair(wa[w], 3, ca);
                 const uint32_t b0 = dequant_pair(wb[w], 0, cb), b1 = dequant_pair(wb[w], 1, cb);
                 const uint32_t b2 = dequant_pair(wb[w], 2, cb), b3 = dequant_pair(wb[w], 3, cb);
-                mma_bf16_16816(acc, a0, b0, a1, b1, xv[w].x, xv[w].y);
-                mma_bf16_16816(acc, a2, b2, a3, b3, xv[w].z, xv[w].w);
-            }
 #pragma unroll
-            for (int w = 0; w < 4; ++w) xv[w] = xn[w];
+                for (int mt = 0; mt < MT; ++mt) {
+                    mma_bf16_16816(acc[mt], a0, b0, a1, b1, xv[mt][w].x, xv[mt][w].y);
+                    mma_bf16_16816(acc[mt], a2, b2, a3, b3, xv[mt][w].z, xv[mt][w].w);
+                }
+            }
+        }
+    }
+    if (!ok) {
+        // a box never landed: record it, wait (bounded) for the copies this warp
+        // still has in flight, and leave the tile unwritten
+        if (lane == 0) {
+            atomicCAS(err, 0, kErrGemvWait);
+            for (int j = i; j < nbw && j < i + kStages; ++j)
+                if (!wait_box(bar0 + 8 * (j % kStages), (uint32_t)(j / kStages) & 1u)) atomicCAS(err, 0, kErrGemvDrain);
         }
     }
 
 #pragma unroll
-    for (int i = 0; i < 4; ++i) red[warp][lane][i] = acc[i];
-    __syncthreads();
-    if (warp == 0) {
-        float sm[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
+        for (int e = 0; e < 4; ++e) red[warp][lane][4 * mt + e] = acc[mt][e];
+    const int all_ok = __syncthreads_and(ok ? 1 : 0);
+    if (warp == 0 && all_ok) {
+        const int rA = r0 + g, rB = rA + 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sm[i] += red[w][lane][i];
-        const int m0 = 2 * t, m1 = 2 * t + 1;    // tokens of c0/c2 and c1/c3
-        if (okA && m0 < M) Y[(size_t)m0 * N + rA] = __float2bfloat16_rn(sm[0]);
-        if (okA && m1 < M) Y[(size_t)m1 * N + rA] = __float2bfloat16_rn(sm[1]);
-        if (okB && m0 < M) Y[(size_t)m0 * N + rB] = __float2bfloat16_rn(sm[2]);
-        if (okB && m1 < M) Y[(size_t)m1 * N + rB] = __float2bfloat16_rn(sm[3]);
+        for (int mt = 0; mt < MT; ++mt) {
+            float sm[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sm[e] += red[w][lane][4 * mt + e];
+            const int m0 = 8 * mt + 2 * t, m1 = m0 + 1;   // tokens of c0/c2 and c1/c3
+            if (rA < N && m0 < M) Y[(size_t)m0 * N + rA] = __float2bfloat16_rn(sm[0]);
+            if (rA < N && m1 < M) Y[(size_t)m1 * N + rA] = __float2bfloat16_rn(sm[1]);
+            if (rB < N && m0 < M) Y[(size_t)m0 * N + rB] = __float2bfloat16_rn(sm[2]);
+            if (rB < N && m1 < M) Y[(size_t)m1 * N + rB] = __float2bfloat16_rn(sm[3]);
+        }
     }
 }
 
-template <int G, int MODE>
-cudaError_t launch_g_mode(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
-                          const void *scales, const uint32_t *qzeros, void *Y, cudaStream_t stream)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+template <int G, int MODE, int MT>
+cudaError_t launch_g(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
+                     const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
 {
     const int64_t blocks = (N + 15) / 16;       // one 16-channel tile per CTA
-    gemv_kernel<G, MODE><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-        (const uint4 *)X, (int)M, (int)N, (int)K, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
-        (__nv_bfloat16 *)Y);
+    gemv_kernel<G, MODE, MT><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+        map, (const uint4 *)X, (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros,
+        (__nv_bfloat16 *)Y, err);
     return cudaGetLastError();
+}
+
+template <int MT>
+cudaError_t launch_mt(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
+                      const uint32_t *qzeros, int group, int mode, void *Y, int *err, cudaStream_t stream)
+{
+    switch (group * 2 + mode) {
+    case 32 * 2 + W4_SYM: return launch_g<32, W4_SYM, MT>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    case 32 * 2 + W4_ASYM: return launch_g<32, W4_ASYM, MT>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    case 64 * 2 + W4_SYM: return launch_g<64, W4_SYM, MT>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    case 64 * 2 + W4_ASYM: return launch_g<64, W4_ASYM, MT>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    case 128 * 2 + W4_SYM: return launch_g<128, W4_SYM, MT>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    case 128 * 2 + W4_ASYM: return launch_g<128, W4_ASYM, MT>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -229,15 +353,22 @@ cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const ui
                         const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                         cudaStream_t stream)
 {
-    switch (group * 2 + mode) {
-    case 32 * 2 + W4_SYM: return launch_g_mode<32, W4_SYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
-    case 32 * 2 + W4_ASYM: return launch_g_mode<32, W4_ASYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
-    case 64 * 2 + W4_SYM: return launch_g_mode<64, W4_SYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
-    case 64 * 2 + W4_ASYM: return launch_g_mode<64, W4_ASYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
-    case 128 * 2 + W4_SYM: return launch_g_mode<128, W4_SYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
-    case 128 * 2 + W4_ASYM: return launch_g_mode<128, W4_ASYM>(X, M, N, K, qweight, scales, qzeros, Y, stream);
-    default: return cudaErrorInvalidValue;
-    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    int *err = device_error_word();
+    if (!err) return cudaErrorUnknown;
+    // the codes as a 2-D array of 32-bit words [N][K/8]; one box = 16 channels x 32 words
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+    const cuuint64_t gstride[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t box[2] = {32u, 16u};
+    const cuuint32_t estride[2] = {1u, 1u};
+    const CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(qweight), gdim, gstride,
+                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    if (M <= 8) return launch_mt<1>(map, X, M, N, K, scales, qzeros, group, mode, Y, err, stream);
+    return launch_mt<2>(map, X, M, N, K, scales, qzeros, group, mode, Y, err, stream);
 }
 
 }  // namespace w4

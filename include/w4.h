@@ -117,9 +117,10 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
  *   workspace, workspace_bytes: device scratch of at least
  *            w4a16_workspace_bytes(M, N, K, group) bytes (may be NULL when
  *            that is 0); 256-byte aligned.
- * Paths: M <= 8 runs the register GEMV (mma.sync from dequantized registers);
- * larger M runs the tcgen05 kernel (dequantized weights in tensor memory,
- * activations in shared memory, fp32 accumulation in tensor memory).
+ * Paths: M <= 16 runs the GEMV (codes streamed to shared memory by TMA,
+ * dequantized in registers, mma.sync); larger M runs the tcgen05 kernel
+ * (dequantized weights in tensor memory, activations in shared memory, fp32
+ * accumulation in tensor memory).
  */
 w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                      const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,

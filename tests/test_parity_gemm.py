@@ -52,11 +52,11 @@ def check(Y, W, X, g, mode):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 13, 16])
 @pytest.mark.parametrize("g", [32, 64, 128])
 @pytest.mark.parametrize("mode", [SYM, ASYM])
 def test_gemv_small_ragged_shapes(w4, M, g, mode):
-    # N not a multiple of the 16-channel tile, K not a multiple of the 512-wide super-chunk
+    # N not a multiple of the 16-channel tile, K not a multiple of the 256-wide k-box
     N, K = 200, 640 if g != 128 else 1152
     W = synth.weights(M + g, N, K, 0.02, 0.01, 5.0)
     X = synth.activations(M + g, M, K, 0.01, 40.0)
@@ -87,7 +87,8 @@ def test_decode_workload_full(w4, prob):
 
 
 TC_SHAPES = [  # (M, N, K): every token-tile width, channels not a multiple of 128, split-K for few tiles
-    (9, 300, 1024), (16, 256, 4096), (17, 130, 2048), (32, 512, 1024), (33, 384, 640), (64, 200, 4096),
+    # (M <= 16 runs the GEMV's two-token-group kernel, M >= 17 the tensor-core kernel)
+    (9, 300, 1024), (16, 256, 4096), (17, 130, 2048), (20, 300, 1024), (24, 256, 4096), (32, 512, 1024), (33, 384, 640), (64, 200, 4096),
     (100, 256, 512), (128, 128, 8192), (129, 640, 1024), (256, 384, 1024), (300, 256, 640), (512, 1024, 1024),
 ]
 
@@ -115,7 +116,7 @@ def test_tc_k_tail(w4, M):
 def test_tc_workspace_is_left_zeroed_and_reusable(w4):
     """Split-K calls leave their counters zeroed: the same workspace serves repeated calls."""
     import torch
-    M, N, K = 16, 256, 4096
+    M, N, K = 24, 256, 4096                      # M > 16: the tensor-core path, split over k
     need = w4.w4a16_workspace_bytes(M, N, K, 128)
     assert need > 0
     W = synth.weights(91, N, K, 0.02)
