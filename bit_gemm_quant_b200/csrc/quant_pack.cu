@@ -7,8 +7,9 @@
 // (blog.freezetheflame.cc quantization deep dive) section 5.3 the offline fold
 // W * s.  The exact arithmetic is spelled out in include/w4.h.
 //
-// Design (HBM-bound stream: 2 B read + about 0.5 B written per weight, a
-// budget of roughly 0.4 warp instructions per weight at full bandwidth):
+// Design (HBM-bound stream: 2 B read + about 0.5 B written per weight; the
+// SMs' issue budget at full bandwidth is about 11 instructions per weight, so
+// the per-weight work is kept to a handful of instructions):
 //   * one resident wave of CTAs; warp w quantizes rows w, w + nwarps, ... as a
 //     stream of 1024-weight items and loads the next item (across row ends)
 //     before it processes the current one; a lane owns 32 consecutive weights,
@@ -16,20 +17,22 @@
 //     with two 32-byte loads; when a warp starts a row it asks L2 to fetch
 //     its next row (cp.async.bulk.prefetch), so HBM latency overlaps a whole
 //     row of work;
-//   * group amax / min / max: 32 in-lane comparisons and at most two
+//   * group amax / min / max: packed bf16x2 min and max over the lane's raw
+//     words (fp32 comparisons after the fold) and at most two
 //     __shfl_xor_sync steps; the per-group IEEE divisions (scale and zero
-//     point) and the reciprocal are then amortized over 32 weights per lane;
-//   * per weight the code is rint(w'/s16) with IEEE semantics: the quotient
-//     is approximated as t = w' * rcp(s16); adding the magic constant
-//     1.5*2^23 + zp leaves 0x4B400000 + u in the float's bits.  If every t of
-//     the lane is further than 2^-16 from a half-integer (the approximation
-//     error is below 5 * 2^-20) those codes equal the codes of the exact
-//     quotient (a lane takes the exact path with probability ~1e-3);
-//     otherwise the lane recomputes its 32 codes with correctly rounded
-//     division (__fdiv_rn).  No lower clamp is needed (the group minimum maps
-//     to -zp exactly) and in symmetric mode no clamp at all (|t| <= 7 * (1 +
-//     2^-11)); groups whose fp16 scale saturated or is subnormal take the
-//     exact path;
+//     point) and the reciprocal are amortized over 32 weights per lane;
+//   * per weight the code is rint(w'/s16) with IEEE semantics.  The fast path
+//     adds the magic constant 1.5*2^23 + zp to w' * rcp(s16), which leaves
+//     0x4B400000 + u in the float's bits, and computes the exact residual
+//     rho = w' - r * s16 (Sterbenz: r * s16 has <= 16 significant bits), two
+//     weights per fma/add instruction.  A pair whose |rho| reaches s16/2 -- an
+//     exact tie of the quotient (common with bf16 weights) or a rounding the
+//     approximation got wrong -- is flagged and recomputed exactly from the
+//     raw words parked in shared memory (ties to even); groups whose fp16
+//     scale saturated or is subnormal take an IEEE-division path;
+//   * y is monotonic in w', so the asymmetric clamp to [0, 15] (needed before
+//     packing: a code of -1 or 16 would borrow from or carry into the next
+//     nibble) runs only in warps where some group's extremes map outside;
 //   * packing: with bits(y) = C + u (C's low byte 0), one IMAD y_b*16 + y_a
 //     puts the byte u_a | u_b << 4 in the low byte; three PRMTs assemble the
 //     word (even elements in the low half-word), and each lane stores its 4
@@ -81,13 +84,91 @@ __device__ __forceinline__ uint32_t pack_word(const uint32_t *y)
 
 __host__ __device__ constexpr int nibble_shift(int e) { return (e & 1) ? 16 + 4 * (e >> 1) : 4 * (e >> 1); }
 
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// The two weights of raw word v (elements 2p and 2p+1 of the lane), folded.
+template <bool FOLD>
+__device__ __forceinline__ float2 weight_pair(uint32_t v, float2 sp)
+{
+    const float2 w = make_float2(bf16lo_to_f32(v), bf16hi_to_f32(v));
+    return FOLD ? __fmul2_rn(w, sp) : w;
+}
+
+// Fast-path codes of the lane's 32 weights: y = fl(w' * rcp(s16) + magic)
+// holds r + zp (or r + 8) in its low bits, r = rint of the approximate
+// quotient; rho = w' - r * s16 is exact.  Bit p of the returned flags marks the
+// weight pair p if either residual reaches half a step (|rho| >= s16 / 2):
+// exact ties of the quotient and roundings the approximation got wrong.  With
+// CLAMP the asymmetric codes are clamped to [0, 15] before packing (a code of
+// -1 or 16 would borrow from or carry into the neighbouring nibble); without
+// it the caller has shown that every y lies in range.  The arithmetic runs on
+// pairs (fma / add of two fp32 lanes per instruction, each correctly rounded).
+template <int MODE, bool FOLD, bool CLAMP>
+__device__ __forceinline__ uint32_t encode(const uint32_t (&cur)[16], const float2 (&sp)[16], float inv,
+                                           float magic, float d, float hd, float ymax, uint32_t (&wd)[4])
+{
+    const float2 inv2 = make_float2(inv, inv), mg2 = make_float2(magic, magic);
+    const float2 nmg2 = make_float2(-magic, -magic), nd2 = make_float2(-d, -d);
+    uint32_t flags = 0u;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint32_t yb[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int p = 4 * w + j;
+            const float2 x = weight_pair<FOLD>(cur[p], sp[p]);
+            float2 y = __ffma2_rn(x, inv2, mg2);
+            if (MODE == W4_ASYM && CLAMP) {
+                y.x = fmaxf(fminf(y.x, ymax), kMagic);
+                y.y = fmaxf(fminf(y.y, ymax), kMagic);
+            }
+            const float2 r = __fadd2_rn(y, nmg2);
+            const float2 rho = __ffma2_rn(r, nd2, x);
+            if (fmaxf(fabsf(rho.x), fabsf(rho.y)) >= hd) flags |= 1u << p;
+            yb[2 * j] = __float_as_uint(y.x);
+            yb[2 * j + 1] = __float_as_uint(y.y);
+        }
+        wd[w] = pack_word(yb);
+    }
+    return flags;
+}
+
+// The exact code of one weight (its fast-path y recomputed, then the tie or
+// the wrong rounding resolved from the exact residual).
+template <int MODE>
+__device__ __forceinline__ uint32_t exact_code(float x, float inv, float magic, float d, float hd, float ymax, int zp)
+{
+    float y = __fmaf_rn(x, inv, magic);
+    if (MODE == W4_ASYM) y = fmaxf(fminf(y, ymax), kMagic);
+    const float r = __fsub_rn(y, magic);
+    const float rho = __fmaf_rn(-r, d, x);
+    const float ar = fabsf(rho);
+    // beyond half a step, or an exact tie with r odd: one step toward rho
+    const int odd = (int)(__float_as_uint(y) ^ (uint32_t)zp) & 1;
+    int q = (int)r;
+    if (ar > hd || (ar == hd && odd)) q += (rho > 0.f) ? 1 : -1;
+    return (MODE == W4_SYM) ? (uint32_t)(min(max(q, -8), 7) + 8) : (uint32_t)min(max(q + zp, 0), 15);
+}
+
 template <int G, int MODE, bool FOLD>
 __global__ void __launch_bounds__(256, 3)
 quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float4 *__restrict__ s,
                   uint4 *__restrict__ qweight, unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros)
 {
     constexpr int LPG = G / 32;                 // lanes per group
-    __shared__ uint4 stash[256 * 4];            // 64 bytes per thread, used only to fix flagged codes
+    __shared__ uint4 stash[4][256];             // raw words, [quarter][thread]: for the rare exact fix
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -97,7 +178,8 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
 
     // The warp's work is the stream of (row, 1024-weight chunk) items of rows
     // warp0, warp0 + nwarps, ...; the next item is loaded before the current
-    // one is processed, across row boundaries.
+    // one is processed, across row boundaries.  Lanes past the end of a row
+    // keep zero words (they are not stored).
     int64_t n = warp0, c0 = 0;
     uint32_t cur[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     if (n < N && lane < KC) {
@@ -119,40 +201,39 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
         {
             const int64_t c = c0 + lane;        // this lane's chunk
             const bool valid = c < KC;
-            {   // this lane's raw words, for the rare exact fix below
-                uint4 *slot = stash + threadIdx.x * 4;
-                slot[0] = make_uint4(cur[0], cur[1], cur[2], cur[3]);
-                slot[1] = make_uint4(cur[4], cur[5], cur[6], cur[7]);
-                slot[2] = make_uint4(cur[8], cur[9], cur[10], cur[11]);
-                slot[3] = make_uint4(cur[12], cur[13], cur[14], cur[15]);
-            }
-            float x[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t v = valid ? cur[i] : 0u;
-                x[2 * i] = bf16lo_to_f32(v);
-                x[2 * i + 1] = bf16hi_to_f32(v);
-            }
-            if (FOLD && valid) {                // w' = fl32(w * s[k])
+            for (int q = 0; q < 4; ++q)
+                stash[q][threadIdx.x] = make_uint4(cur[4 * q], cur[4 * q + 1], cur[4 * q + 2], cur[4 * q + 3]);
+            float2 sp[16];                      // smoothing factors of the weight pairs
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 f = __ldg(s + 8 * c + i);
-                    x[4 * i] = __fmul_rn(x[4 * i], f.x);
-                    x[4 * i + 1] = __fmul_rn(x[4 * i + 1], f.y);
-                    x[4 * i + 2] = __fmul_rn(x[4 * i + 2], f.z);
-                    x[4 * i + 3] = __fmul_rn(x[4 * i + 3], f.w);
-                }
+            for (int i = 0; i < 8; ++i) {
+                const float4 f = (FOLD && valid) ? __ldg(s + 8 * c + i) : make_float4(1.f, 1.f, 1.f, 1.f);
+                sp[2 * i] = make_float2(f.x, f.y);
+                sp[2 * i + 1] = make_float2(f.z, f.w);
             }
 
             // ---- group statistics, scale and zero-point ----
-            float d, inv, magic, hi = 0.f;
+            float lmin, lmax;                   // extremes of this lane's 32 weights w'
+            if (!FOLD) {                        // on the raw bf16 pairs: one min and one max per pair
+                uint32_t pmin = cur[0], pmax = cur[0];
+#pragma unroll
+                for (int i = 1; i < 16; ++i) { pmin = bmin2(pmin, cur[i]); pmax = bmax2(pmax, cur[i]); }
+                lmin = fminf(bf16lo_to_f32(pmin), bf16hi_to_f32(pmin));
+                lmax = fmaxf(bf16lo_to_f32(pmax), bf16hi_to_f32(pmax));
+            } else {
+                lmin = lmax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 x = weight_pair<true>(cur[i], sp[i]);
+                    lmin = fminf(lmin, fminf(x.x, x.y));
+                    lmax = fmaxf(lmax, fmaxf(x.x, x.y));
+                }
+            }
+            float d, mn = 0.f, mx = 0.f, hi = 0.f;
             int zp;
             unsigned short s16;
-            bool exact_only;
             if (MODE == W4_SYM) {
-                float a = 0.f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+                float a = fmaxf(fabsf(lmin), fabsf(lmax));
 #pragma unroll
                 for (int off = LPG / 2; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
                 const float s32 = __fdiv_rn(a, 7.0f);
@@ -160,9 +241,8 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
                 d = __half2float(__ushort_as_half(s16));
                 zp = 8;
             } else {
-                float mn = 0.f, mx = 0.f;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
+                mn = fminf(0.f, lmin);
+                mx = fmaxf(0.f, lmax);
 #pragma unroll
                 for (int off = LPG / 2; off > 0; off >>= 1) {
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -175,62 +255,43 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
                 hi = (float)(15 - zp);
             }
             // the fast path assumes a normal, unsaturated fp16 scale (or a zero one)
-            exact_only = (s16 == 0x7BFF) || (d > 0.f && d < 6.103515625e-05f);
-            inv = (d > 0.f) ? rcp_approx(d) : 0.f;
-            magic = kMagic + (float)zp;         // exact: 1.5*2^23 + zp < 2^24
+            const bool exact_only = (s16 == 0x7BFF) || (d > 0.f && d < 6.103515625e-05f);
+            const float inv = (d > 0.f) ? rcp_approx(d) : 0.f;
+            const float magic = kMagic + (float)zp;   // exact: 1.5*2^23 + zp < 2^24
+            const float hd = (d > 0.f) ? 0.5f * d : __int_as_float(0x7F800000);
+            const float ymax = magic + hi;
 
             // ---- codes ----
-            // y = fl(w' * rcp(s16) + (1.5*2^23 + zp)) holds r + zp (or r + 8) in its low
-            // bits, r = rint of the approximate quotient.  rho = w' - r*s16 is exact
-            // (Sterbenz; r*s16 has <= 16 bits), so |rho| >= s16/2 flags exactly the
-            // weights whose code needs the exact decision: ties of the exact quotient
-            // (frequent with bf16 weights and short fp16 scales) and roundings the
-            // approximation got wrong.  Those are fixed below, one element index at a
-            // time, only when some lane of the warp has one.
-            const float hd = (d > 0.f) ? 0.5f * d : __int_as_float(0x7F800000);
-            // asymmetric codes are clamped to [0, 15] before packing: a code of -1 (a
-            // weight at the group minimum whose quotient is a tie below -zp) would
-            // borrow from its neighbour nibble in pack_word.  The clamp changes no
-            // result: rint(min/s16) = -zp unless zp was clipped to 15, and the method
-            // clips every code to [0, 15] anyway.
-            const float ymax = magic + hi;
-            uint32_t wd[4], flags = 0u;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                uint32_t yb[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float y = __fmaf_rn(x[8 * w + i], inv, magic);
-                    if (MODE == W4_ASYM) y = fmaxf(fminf(y, ymax), kMagic);
-                    const float r = __fsub_rn(y, magic);
-                    const float rho = __fmaf_rn(-r, d, x[8 * w + i]);
-                    flags |= (fabsf(rho) >= hd) ? (1u << (8 * w + i)) : 0u;
-                    yb[i] = __float_as_uint(y);
-                }
-                wd[w] = pack_word(yb);
-            }
+            // y is monotonic in w', so when the group's extremes mn and mx map into
+            // [0, 15] every weight of the group does and no clamp is needed; the
+            // (rare) warps with a group whose extremes fall outside run the clamped
+            // variant.  Symmetric codes never leave [1, 15]: |w'/s16| <= 7 (1 + 2^-11).
+            uint32_t wd[4], flags;
+            bool clamp = false;
+            if (MODE == W4_ASYM)
+                clamp = __fmaf_rn(mn, inv, magic) < kMagic || __fmaf_rn(mx, inv, magic) > ymax;
+            if (MODE == W4_ASYM && __any_sync(0xffffffffu, clamp))
+                flags = encode<MODE, FOLD, true>(cur, sp, inv, magic, d, hd, ymax, wd);
+            else
+                flags = encode<MODE, FOLD, false>(cur, sp, inv, magic, d, hd, ymax, wd);
             if (__any_sync(0xffffffffu, flags != 0u)) {
-                // rare path: fix the flagged codes one by one from the raw bf16 words
-                // parked in this lane's shared-memory slot (no live fp32 copies)
-                const uint32_t *raw = (const uint32_t *)(stash + threadIdx.x * 4);
+                // fix the flagged pairs from the raw words parked in shared memory
+                // (a warp has one in about two items with bf16 weights: exact ties
+                // are common when the fp16 scale has few significant bits)
                 uint32_t m = flags;
                 while (m) {
-                    const int i = __ffs(m) - 1;
+                    const int p = __ffs(m) - 1;
                     m &= m - 1u;
-                    float xi = (i & 1) ? bf16hi_to_f32(raw[i >> 1]) : bf16lo_to_f32(raw[i >> 1]);
-                    if (FOLD) xi = __fmul_rn(xi, __ldg((const float *)s + 32 * c + i));
-                    float y = __fmaf_rn(xi, inv, magic);
-                    if (MODE == W4_ASYM) y = fmaxf(fminf(y, ymax), kMagic);
-                    const float r = __fsub_rn(y, magic);
-                    const float rho = __fmaf_rn(-r, d, xi);
-                    // beyond half a step, or an exact tie with r odd: one step toward rho
-                    const int odd = (int)(__float_as_uint(y) ^ (uint32_t)zp) & 1;
-                    int q = (int)r;
-                    if (fabsf(rho) > hd || odd) q += (rho > 0.f) ? 1 : -1;
-                    const int u = (MODE == W4_SYM) ? min(max(q, -8), 7) + 8 : min(max(q + zp, 0), 15);
-                    const int e = i & 7, sh = (e & 1) ? 16 + 4 * (e >> 1) : 4 * (e >> 1);
-                    const uint32_t keep = ~(0xFu << sh), val = (uint32_t)u << sh;
-                    const int w = i >> 3;
+                    const uint32_t v = ((const uint32_t *)&stash[p >> 2][threadIdx.x])[p & 3];
+                    float2 sv = make_float2(1.f, 1.f);
+                    if (FOLD) sv = __ldg((const float2 *)s + 16 * c + p);
+                    const float2 x = weight_pair<FOLD>(v, sv);
+                    const uint32_t u0 = exact_code<MODE>(x.x, inv, magic, d, hd, ymax, zp);
+                    const uint32_t u1 = exact_code<MODE>(x.y, inv, magic, d, hd, ymax, zp);
+                    // elements 2p, 2p+1: nibble (p & 3) of the low and of the high half-word
+                    const int sh = 4 * (p & 3), w = p >> 2;
+                    const uint32_t keep = ~((0xFu << sh) | (0xFu << (16 + sh)));
+                    const uint32_t val = (u0 << sh) | (u1 << (16 + sh));
                     wd[0] = (w == 0) ? ((wd[0] & keep) | val) : wd[0];
                     wd[1] = (w == 1) ? ((wd[1] & keep) | val) : wd[1];
                     wd[2] = (w == 2) ? ((wd[2] & keep) | val) : wd[2];
@@ -241,12 +302,16 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
             if (exact_only) {                   // saturated or subnormal scale: IEEE division
                 uint32_t wx[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float q = rintf(__fdiv_rn(x[i], d));
-                    int u;
-                    if (MODE == W4_SYM) u = (int)fminf(fmaxf(q, -8.f), 7.f) + 8;
-                    else u = (int)fminf(fmaxf(q + (float)zp, 0.f), 15.f);
-                    wx[i >> 3] |= (uint32_t)u << nibble_shift(i & 7);
+                for (int p = 0; p < 16; ++p) {
+                    const float2 x = weight_pair<FOLD>(cur[p], sp[p]);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float q = rintf(__fdiv_rn(h ? x.y : x.x, d));
+                        int u;
+                        if (MODE == W4_SYM) u = (int)fminf(fmaxf(q, -8.f), 7.f) + 8;
+                        else u = (int)fminf(fmaxf(q + (float)zp, 0.f), 15.f);
+                        wx[p >> 2] |= (uint32_t)u << nibble_shift(2 * (p & 3) + h);
+                    }
                 }
                 out = make_uint4(wx[0], wx[1], wx[2], wx[3]);
             }
