@@ -14,11 +14,14 @@ every activation batch is multiplied by its packed weight (w4a16_gemm).
                     value = GEMM TFLOP/s over the step
   quantizer         W[28672, 8192]: g in {32,64,128} x {sym, asym} + smoothing fold
 
-The K timed steps are captured in one CUDA graph and replayed once between
-CUDA events on the launching stream; event-record nodes between the kernels
-give each kernel's device time inside that same replay.  Inputs rotate over
+The K timed steps are captured in one CUDA graph (kernel nodes only) and
+replayed once between CUDA events on the launching stream.  Inputs rotate over
 two sets so that no kernel finds its inputs in the 126 MB L2: each GEMM reads
 the weights packed one step earlier, after more than 126 MB of other traffic.
+Each kernel's device time is measured the same way, live, from a graph of K
+launches of that kernel alone over enough copies of its inputs (> 2x L2) that
+every launch reads them from HBM.  (An event-record node between kernels
+inside the step graph would cost several microseconds per kernel.)
 
 Under torchrun (N > 1) every rank runs its own replica with its own seeds
 (weak scaling, no collective on the data path); the timed region is bracketed
@@ -29,7 +32,6 @@ the same workload instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
-import ctypes
 import hashlib
 import json
 import os
@@ -114,41 +116,6 @@ def kernel_name(M: int) -> str:
 class Launch:
     def __init__(self, name, work_bytes, flops, label):
         self.name, self.bytes, self.flops, self.label = name, work_bytes, flops, label
-
-
-# ------------------------------------------------------------ cudart ----
-
-class CudaRT:
-    """The few runtime calls torch does not expose: external event-record
-    nodes inside a captured graph, and their elapsed times."""
-
-    def __init__(self):
-        self.L = ctypes.CDLL("libcudart.so.12")
-        self.L.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_uint]
-        self.L.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
-        self.L.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
-        self.L.cudaEventDestroy.argtypes = [ctypes.c_void_p]
-
-    def _check(self, rc, what):
-        if rc != 0:
-            raise RuntimeError("%s failed with cudaError %d" % (what, rc))
-
-    def event(self):
-        ev = ctypes.c_void_p()
-        self._check(self.L.cudaEventCreateWithFlags(ctypes.byref(ev), 0), "cudaEventCreateWithFlags")
-        return ev
-
-    def record_external(self, ev, stream_handle: int):
-        self._check(self.L.cudaEventRecordWithFlags(ev, ctypes.c_void_p(stream_handle), 1),
-                    "cudaEventRecordWithFlags")
-
-    def elapsed_ms(self, a, b) -> float:
-        ms = ctypes.c_float()
-        self._check(self.L.cudaEventElapsedTime(ctypes.byref(ms), a, b), "cudaEventElapsedTime")
-        return float(ms.value)
-
-    def destroy(self, ev):
-        self.L.cudaEventDestroy(ev)
 
 
 # ------------------------------------------------------------ clocks ----
@@ -303,20 +270,13 @@ def run_w4(args, rank, world, local_rank):
                 launches.append(Launch(kernel_name(pp.M), roofline.gemm_bytes(pp.M, pp.N, pp.K, pp.group, pp.mode),
                                        roofline.gemm_flops(pp.M, pp.N, pp.K), pp.name))
 
-    def step(si, marks=None, rt=None, stream_handle=None):
+    def step(si):
         r, r_prev = si % R, (si + 1) % R
-        i = 0
         for k in keys:
             p = qp[k]
-            if marks is not None:
-                rt.record_external(marks[i], stream_handle)
-            i += 1
             w4.quant_pack(W_d[k][r], p.group, p.mode, s=s_d[k], out=packed[k][r])
             for key, pp in plist:
                 if key == k and pp.M > 0:
-                    if marks is not None:
-                        rt.record_external(marks[i], stream_handle)
-                    i += 1
                     q, sc, z = packed[k][r_prev]
                     w4.gemm(X_d[pp.name][r], q, sc, z, pp.group, pp.mode, N=pp.N, workspace=ws_d[pp.name],
                             out=Y_d[pp.name])
@@ -327,18 +287,16 @@ def run_w4(args, rank, world, local_rank):
         step(si)
     torch.cuda.synchronize()
 
-    # ---- capture the K timed steps with event nodes between kernels ----
-    rt = CudaRT()
+    # ---- capture the K timed steps: kernels only, no nodes between them ----
+    # (an event-record node inside a graph costs several microseconds, so the
+    # per-kernel durations are taken from separate graphs below)
     K = args.steps
-    marks = [rt.event() for _ in range(K * per_step + 1)]
     graph = torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream(device)
     cap_stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.graph(graph, stream=cap_stream):
-        h = torch.cuda.current_stream().cuda_stream
         for si in range(K):
-            step(si, marks[si * per_step:(si + 1) * per_step], rt, h)
-        rt.record_external(marks[-1], h)
+            step(si)
     torch.cuda.synchronize()
 
     # ---- sustained load (untimed) so the clock samples cover a steady state ----
@@ -375,14 +333,57 @@ def run_w4(args, rank, world, local_rank):
         sampler.mark_end()
         clocks = sampler.stop()
         clocks["remeasured"] = True
+    del graph
 
-    # per-kernel device time inside this replay
+    # ---- per-kernel device time: each launch of the step alone, K times in one
+    # graph, over enough copies of its inputs (> 2x L2) that every launch reads
+    # them from HBM; CUDA events on the launching stream around the replay ----
+    L2_BYTES = 126 << 20
+
+    def kernel_graph_ms(fns):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(device)
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=cs):
+            for i in range(K):
+                fns[i % len(fns)]()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(cs):
+            e0.record(cs)
+            g.replay()
+            e1.record(cs)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / K
+        del g
+        return ms
+
+    def copies(ts, nbytes):
+        n = max(2, -(-2 * L2_BYTES // max(nbytes, 1)))
+        return [tuple(None if t is None else t.clone() for t in ts) for _ in range(n)]
+
     kt = {}
-    for si in range(K):
-        for j, L in enumerate(launches):
-            a = marks[si * per_step + j]
-            b = marks[si * per_step + j + 1]
-            kt.setdefault((L.name, L.label), []).append(rt.elapsed_ms(a, b))
+    for k in keys:
+        p = qp[k]
+        W_pool = copies((W_d[k][0],), W_d[k][0].numel() * 2)
+        out = packed[k][0]
+        fns = [(lambda Wc=Wc: w4.quant_pack(Wc[0], p.group, p.mode, s=s_d[k], out=out)) for Wc in W_pool]
+        kt[("w4_quant_pack", k)] = kernel_graph_ms(fns)
+        del W_pool
+        for key, pp in plist:
+            if key == k and pp.M > 0:
+                q0, sc0, z0 = packed[k][0]
+                nb = q0.numel() * 4 + sc0.numel() * 2 + (0 if z0 is None else z0.numel() * 4)
+                P_pool = copies((q0, sc0, z0), nb)
+                fns = [(lambda Pc=Pc, pp=pp: w4.gemm(X_d[pp.name][0], Pc[0], Pc[1], Pc[2], pp.group, pp.mode,
+                                                     N=pp.N, workspace=ws_d[pp.name], out=Y_d[pp.name]))
+                       for Pc in P_pool]
+                kt[(kernel_name(pp.M), pp.name)] = kernel_graph_ms(fns)
+                del P_pool
+    torch.cuda.synchronize()
 
     step_bytes = sum(L.bytes for L in launches)
     step_flops = sum(L.flops for L in launches)
@@ -400,8 +401,8 @@ def run_w4(args, rank, world, local_rank):
     kernels = {}
     by_name = {}
     for L in launches:
-        ts = kt[(L.name, L.label)]
-        avg = statistics.mean(ts)
+        avg = kt[(L.name, L.label)]
+        ts = [avg] * K
         ent = {"launches": len(ts), "avg_us": round(avg * 1e3, 3), "bytes": L.bytes,
                "gbs": round(L.bytes / (avg * 1e-3) / 1e9, 1),
                "hbm_frac": round(L.bytes / (avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
@@ -446,9 +447,6 @@ def run_w4(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.workload, plist, keys, qp, host_W, host_X, host_s, args.cpu_budget)
 
-    for ev in marks:
-        rt.destroy(ev)
-    del graph
     if rank == 0:
         wl_desc = {
             "decode": "decode GEMV: M=1, K=4096, N in {4096,11008,12288}, asymmetric INT4 g=128, fp16 scales, uint4 zero-points; step = w4_quant_pack + w4a16_gemm per layer",
@@ -458,12 +456,12 @@ def run_w4(args, rank, world, local_rank):
         }[args.workload]
         out = {
             "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K,
-            "warmup": max(3, args.warmup) + replays, "ms_per_step": round(max_ms / K, 5),
+            "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / K, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": wl_desc, "codes": "int4 packed 8 per uint32", "accumulate": "fp32",
                        "l2": "inputs rotate over 2 sets; each kernel's inputs were last touched before >126 MB of other traffic",
-                       "timing": "K steps captured in one CUDA graph, replayed between CUDA events on the launching stream; max over ranks",
+                       "timing": "K steps captured in one CUDA graph (kernels only), replayed between CUDA events on the launching stream after %d untimed replays; max over ranks; per-kernel durations from a graph of K launches of that kernel alone over rotating input copies (> 2x L2), between CUDA events on its stream" % replays,
                        "parallelism": "replicas (dp%d), no data-path collective" % world},
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": K * per_step * world, "clocks": clocks,

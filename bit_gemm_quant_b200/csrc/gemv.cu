@@ -19,8 +19,8 @@
 //     takes the 256-wide k-boxes w, w+4, w+8, ... and the four partial tiles
 //     are summed in shared memory at the end (no global scratch);
 //   * the codes stream HBM -> shared memory by TMA (one 2-D box of 16 rows x
-//     128 bytes per k-box, 128-byte swizzle), three boxes in flight per warp on
-//     the warp's own mbarrier ring, so a resident CTA keeps 24 KB of reads
+//     128 bytes per k-box, 128-byte swizzle), four boxes in flight per warp on
+//     the warp's own mbarrier ring, so a resident CTA keeps 32 KB of reads
 //     outstanding and the loads cost the warps one instruction per box;
 //   * per k-box, each lane turns one (channel, group) scale and zero-point into
 //     the bf16x2 constants below and parks them in the warp's shared-memory
@@ -44,7 +44,8 @@
 //     words, and the activation fragment for token g is then the plain 16-byte
 //     chunk of X[g] at the word's k;
 //   * tokens occupy the MMA's N = 8 columns, MT groups of 8 tokens (M <= 8 * MT);
-//     lanes whose token is >= M feed zeros.
+//     lanes whose token is >= M repeat token M-1 into MMA columns that are
+//     never stored.
 // Every wait on an mbarrier is bounded in time; a wait that runs out records
 // an error code (read by w4_device_error), and the warp stops computing, waits
 // (again bounded) for its own copies in flight and returns.
@@ -56,7 +57,7 @@ namespace w4 {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr int kStages = 3;                       // k-boxes in flight per warp
+constexpr int kStages = 4;                       // k-boxes in flight per warp
 constexpr int kBoxK = 256;                       // k per box: 32 words of 8 codes
 constexpr int kBoxBytes = 16 * 128;              // 16 channels x 128 bytes
 constexpr uint64_t kWaitLimitNs = 200000000ull;  // 200 ms; a box lands in microseconds
@@ -144,13 +145,8 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const uint4 
     return bf2_fma(D, gc.x, bf2_mul(D, gc.y));
 }
 
-__device__ __forceinline__ uint4 ldg_x(const uint4 *p, bool ok)
-{
-    return ok ? __ldg(p) : make_uint4(0u, 0u, 0u, 0u);
-}
-
 template <int G, int MODE, int MT>
-__global__ void __launch_bounds__(kWarps * 32, 6)
+__global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 6 : 4)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
             __nv_bfloat16 *__restrict__ Y, int *err)
@@ -209,9 +205,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
     };
     if (nbw > 0) load_consts(0);
 
-    float acc[MT][4];
+    // two accumulator sets (the first and the second MMA of every word pair)
+    // halve the dependent chain of MMAs
+    float acc[MT][4], acc2[MT][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[mt][e] = acc2[mt][e] = 0.f;
 
     bool ok = true;
     int i = 0;
@@ -242,8 +242,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int c = t + 4 * h;             // chunk of this half
-            const int k0 = b * kBoxK + c * 32;   // first k of the chunk
-            const bool kin = k0 < K;             // K is a multiple of 32: chunks are whole
+            // first k of the chunk; a chunk past the end of K (K is a multiple of
+            // 32, chunks are whole) reads the last chunk's activations instead:
+            // its codes are zero-filled by TMA and its groups' constants have
+            // s16 = 0, so every w^ there is 0 and the activations only need to
+            // be finite
+            const int k0 = min(b * kBoxK + c * 32, K - 32);
             const uint4 ca = sconst[warp][(g) + 16 * ((c * 32) / G)];
             const uint4 cb = sconst[warp][(g + 8) + 16 * ((c * 32) / G)];
             const uint4 wa4 = h ? qa1 : qa0, wb4 = h ? qb1 : qb0;
@@ -252,10 +256,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
             uint4 xv[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const int tok = g + 8 * mt;
-                const uint4 *xrow = X + ((size_t)(tok < M ? tok : 0) * K + k0) / 8;
+                // a token past M reads token M-1: its MMA column is never stored
+                const int tok = min(g + 8 * mt, M - 1);
+                const uint4 *xrow = X + ((size_t)tok * K + k0) / 8;
 #pragma unroll
-                for (int w = 0; w < 4; ++w) xv[mt][w] = ldg_x(xrow + w, kin && tok < M);
+                for (int w = 0; w < 4; ++w) xv[mt][w] = __ldg(xrow + w);
             }
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
@@ -266,7 +271,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     mma_bf16_16816(acc[mt], a0, b0, a1, b1, xv[mt][w].x, xv[mt][w].y);
-                    mma_bf16_16816(acc[mt], a2, b2, a3, b3, xv[mt][w].z, xv[mt][w].w);
+                    mma_bf16_16816(acc2[mt], a2, b2, a3, b3, xv[mt][w].z, xv[mt][w].w);
                 }
             }
         }
@@ -284,7 +289,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) red[warp][lane][4 * mt + e] = acc[mt][e];
+        for (int e = 0; e < 4; ++e) red[warp][lane][4 * mt + e] = acc[mt][e] + acc2[mt][e];
     const int all_ok = __syncthreads_and(ok ? 1 : 0);
     if (warp == 0 && all_ok) {
         const int rA = r0 + g, rB = rA + 8;

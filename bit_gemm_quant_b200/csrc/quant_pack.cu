@@ -10,13 +10,13 @@
 // Design (HBM-bound stream: 2 B read + about 0.5 B written per weight; the
 // SMs' issue budget at full bandwidth is about 11 instructions per weight, so
 // the per-weight work is kept to a handful of instructions):
-//   * one resident wave of CTAs; warp w quantizes rows w, w + nwarps, ... as a
-//     stream of 1024-weight items and loads the next item (across row ends)
-//     before it processes the current one; a lane owns 32 consecutive weights,
-//     which always lie in one group (g = 32, 64, 128 is 1, 2 or 4 lanes), read
-//     with two 32-byte loads; when a warp starts a row it asks L2 to fetch
-//     its next row (cp.async.bulk.prefetch), so HBM latency overlaps a whole
-//     row of work;
+//   * one resident wave of CTAs; the matrix is a row-major sequence of
+//     1024-weight items and warp w takes items w, w + nwarps, ..., so the
+//     warps' shares differ by at most one item; a warp loads its next item
+//     before it processes the current one and asks L2 for the one after
+//     (cp.async.bulk.prefetch); a lane owns 32 consecutive weights, which
+//     always lie in one group (g = 32, 64, 128 is 1, 2 or 4 lanes), read with
+//     two 32-byte loads;
 //   * group amax / min / max: packed bf16x2 min and max over the lane's raw
 //     words (fp32 comparisons after the fold) and at most two
 //     __shfl_xor_sync steps; the per-group IEEE divisions (scale and zero
@@ -176,28 +176,44 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
     const int64_t NG = K / G;                   // groups per row
     const int64_t ZW = (NG + 7) >> 3;           // zero-point words per row
 
-    // The warp's work is the stream of (row, 1024-weight chunk) items of rows
-    // warp0, warp0 + nwarps, ...; the next item is loaded before the current
-    // one is processed, across row boundaries.  Lanes past the end of a row
-    // keep zero words (they are not stored).
-    int64_t n = warp0, c0 = 0;
+    // The work is the row-major sequence of 1024-weight items (32 chunks of a
+    // row; the last item of a row may be shorter).  Warp w takes items w,
+    // w + nwarps, w + 2 nwarps, ... (so every warp gets the same number of
+    // items, whatever N and K), loads its next item before it processes the
+    // current one and asks L2 for the item after that.  Lanes past the end of
+    // a row keep zero words (they are not stored).
+    const int64_t IPR = (KC + 31) >> 5;         // items per row
+    const int64_t step_rows = nwarps / IPR, step_items = nwarps % IPR;
+    auto advance = [&](int64_t &row, int64_t &item) {
+        row += step_rows;
+        item += step_items;
+        if (item >= IPR) { item -= IPR; ++row; }
+    };
+    int64_t n = warp0 / IPR, it = warp0 % IPR;  // row and item-in-row of the current item
     uint32_t cur[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    if (n < N && lane < KC) {
-        const uint4 *p = W + n * (K >> 3) + 4 * lane;
+    if (n < N && 32 * it + lane < KC) {
+        const uint4 *p = W + n * (K >> 3) + 4 * (32 * it + lane);
         ld32(p, *(uint32_t(*)[8])&cur[0]);
         ld32(p + 2, *(uint32_t(*)[8])&cur[8]);
     }
     while (n < N) {
-        int64_t nn = n, nc0 = c0 + 32;
-        if (nc0 >= KC) { nc0 = 0; nn += nwarps; }
+        const int64_t c0 = 32 * it;             // first chunk of the current item
+        int64_t nn = n, nit = it;
+        advance(nn, nit);
         uint32_t nxt[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (nn < N && nc0 + lane < KC) {
-            const uint4 *p = W + nn * (K >> 3) + 4 * (nc0 + lane);
+        if (nn < N && 32 * nit + lane < KC) {
+            const uint4 *p = W + nn * (K >> 3) + 4 * (32 * nit + lane);
             ld32(p, *(uint32_t(*)[8])&nxt[0]);
             ld32(p + 2, *(uint32_t(*)[8])&nxt[8]);
         }
-        if (c0 == 0 && lane == 0 && n + nwarps < N)   // the row after this one, HBM -> L2
-            prefetch_l2(W + (n + nwarps) * (K >> 3), (size_t)K * 2);
+        if (lane == 0) {                        // the item after next, HBM -> L2
+            int64_t pn = nn, pit = nit;
+            advance(pn, pit);
+            if (pn < N) {
+                const int64_t pc = 32 * pit, nch = (KC - pc) < 32 ? (KC - pc) : 32;
+                prefetch_l2(W + pn * (K >> 3) + 4 * pc, (size_t)nch * 64);
+            }
+        }
         {
             const int64_t c = c0 + lane;        // this lane's chunk
             const bool valid = c < KC;
@@ -332,7 +348,7 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
 #pragma unroll
         for (int i = 0; i < 16; ++i) cur[i] = nxt[i];
         n = nn;
-        c0 = nc0;
+        it = nit;
     }
 }
 
@@ -347,7 +363,8 @@ cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, u
                                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_pack_kernel<G, MODE, false>, threads, 0);
         if (e != cudaSuccess || per_sm < 1) per_sm = 1;
     }
-    int64_t blocks = (N + 7) / 8;                // one warp per row at most
+    const int64_t items = N * ((K / 32 + 31) / 32);   // 1024-weight items
+    int64_t blocks = (items + 7) / 8;            // one warp per item at most
     const int64_t cap = (int64_t)kNumSMs * per_sm;   // one resident wave; warps stride over rows
     if (blocks > cap) blocks = cap;
     if (s)
