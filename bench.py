@@ -105,7 +105,7 @@ def problems_for(workload: str):
     if workload == "decode":
         return [(p.name, p) for p in probs]
     if workload in ("smallbatch", "prefill"):
-        return [("W", p) for p in probs]
+        return [(workload + "_W", p) for p in probs]
     return [(p.name, p) for p in probs]
 
 

@@ -15,7 +15,7 @@ def test_defaults_and_workloads():
     assert a.gpus == 1 and a.impl == "w4" and a.workload == "decode" and a.warmup >= 3
     keys = [k for k, _ in bench.problems_for("decode")]
     assert len(keys) == 3 and len(set(keys)) == 3
-    assert {k for k, _ in bench.problems_for("prefill")} == {"W"}
+    assert {k for k, _ in bench.problems_for("prefill")} == {"prefill_W"}
 
 
 def test_algorithmic_bytes():
