@@ -210,15 +210,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v)
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
 {
     uint32_t d;
@@ -285,7 +276,9 @@ struct TcCfg {
     // pipeline depth: as many 32-column A stages as fit beside the accumulator, at most 6 (even)
     static constexpr int kStages = ((kCols - BN) / 32 >= 6) ? 6 : 4;
     static constexpr int kACol0 = BN;                                   // A stages follow the BN fp32 accumulator columns
-    static constexpr int kStageBytes = BN * 128;                        // activation box bytes
+    static constexpr int kBBytes = BN * 128;                            // activation box bytes
+    static constexpr int kCodeBytes = 128 * 32;                         // codes box: 128 channels x 64 k
+    static constexpr int kStageBytes = kBBytes + kCodeBytes;            // a multiple of 1024
     static_assert(kACol0 + kStages * 32 <= kCols, "tensor memory overflow");
     static constexpr int kMinBlocks = (BN == 256) ? 1 : 2;
     // kind::f16, fp32 D, bf16 A and B, both K-major, N = BN, M = 128
@@ -293,15 +286,16 @@ struct TcCfg {
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 };
 
+// Scales and zero-points of one channel's two 32-weight halves of a k-block.
 struct SlotData {
-    uint4 w0, w1;
     unsigned short s0, s1;
     uint32_t z0, z1;
 };
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, TcCfg<BN>::kMinBlocks)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, int group_log2, int asym,
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
+               const __grid_constant__ CUtensorMap tmap_y, int y_tma, int M, int N, int K, int group_log2, int asym,
                const uint4 *__restrict__ qweight, const unsigned short *__restrict__ scales,
                const uint32_t *__restrict__ qzeros, __nv_bfloat16 *__restrict__ Y, float *__restrict__ partial,
                unsigned *__restrict__ counters, int splits, int kb_per_split)
@@ -348,6 +342,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_x) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_q) : "memory");
             int issued = 0;
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
@@ -355,6 +350,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
                 if (!wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyTma)) break;
                 mbar_arrive_expect_tx(&full_b[s], C::kStageBytes);
                 tma_load_2d(sB + s * C::kStageBytes, &tmap_x, &full_b[s], (kb_begin + i) * kKB, m0);
+                tma_load_2d(sB + s * C::kStageBytes + C::kBBytes, &tmap_q, &full_b[s], (kb_begin + i) * 8, n0);
                 ++issued;
             }
             // drain: every issued copy must have landed before the CTA may exit
@@ -388,18 +384,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
         const int r = 32 * q + lane;
         const int n = n0 + r;
         const bool okn = n < N;
-        const uint4 *qrow = qweight + (size_t)(okn ? n : 0) * KQ;
         const unsigned short *srow = scales + (size_t)(okn ? n : 0) * NG;
         const uint32_t *zrow = qzeros + (size_t)(okn ? n : 0) * ZW;
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
 
-        constexpr int D = 4;                         // k-blocks prefetched per thread
+        // the codes arrive with the activations (TMA, full_b); only the scales
+        // and zero-points are loaded here, D k-blocks of this warp ahead
+        constexpr int D = 4;
         SlotData buf[D];
         auto fetch = [&](int i, SlotData &sd) {
-            const int kq = (kb_begin + i) * 2;       // first 16-byte chunk of this k-block
-            const bool ok0 = okn, ok1 = okn && (kq + 1 < KQ);
-            sd.w0 = ok0 ? ld_stream(qrow + kq) : make_uint4(0u, 0u, 0u, 0u);
-            sd.w1 = ok1 ? ld_stream(qrow + kq + 1) : make_uint4(0u, 0u, 0u, 0u);
+            const int kq = (kb_begin + i) * 2;       // first 32-weight half of this k-block
+            const bool ok0 = okn && kq < KQ, ok1 = okn && (kq + 1 < KQ);
             const int j0 = (kq * 32) >> group_log2, j1 = ((kq + 1) * 32) >> group_log2;
             sd.s0 = ok0 ? __ldg(srow + j0) : (unsigned short)0;
             sd.s1 = ok1 ? __ldg(srow + j1) : (unsigned short)0;
@@ -420,11 +415,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
             for (int d = 0; d < D; ++d) {
                 const int i = i0 + 2 * d;
                 if (i >= nkb || !ok) break;
+                const int s = i % kStages;
+                const uint32_t ph = (i / kStages) & 1;
+                // full_b also means the MMAs of this stage's previous round are done
+                // (the producer refilled it only after their commit), so its
+                // tensor-memory A columns are free
+                if (!__all_sync(0xffffffffu, wait_bounded(&full_b[s], ph, abort_flag, kErrWaitEmptyDeq))) {
+                    ok = false;
+                    break;
+                }
+                // this channel's 64 codes: 32 bytes of row r of the codes box
+                const uint4 *cs = (const uint4 *)(sB + s * C::kStageBytes + C::kBBytes + r * 32);
+                const uint4 w0 = cs[0], w1 = cs[1];
                 uint32_t v[32];
                 const GroupConst c0 = group_const(buf[d].s0, buf[d].z0);
                 const GroupConst c1 = group_const(buf[d].s1, buf[d].z1);
-                const uint32_t wa[4] = {buf[d].w0.x, buf[d].w0.y, buf[d].w0.z, buf[d].w0.w};
-                const uint32_t wb[4] = {buf[d].w1.x, buf[d].w1.y, buf[d].w1.z, buf[d].w1.w};
+                if (i + 2 * D < nkb) fetch(i + 2 * D, buf[d]);
+                const uint32_t wa[4] = {w0.x, w0.y, w0.z, w0.w};
+                const uint32_t wb[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
                 for (int w = 0; w < 4; ++w)
 #pragma unroll
@@ -432,13 +440,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
                         v[4 * w + j] = dequant_pair(wa[w], j, c0);
                         v[16 + 4 * w + j] = dequant_pair(wb[w], j, c1);
                     }
-                if (i + 2 * D < nkb) fetch(i + 2 * D, buf[d]);
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
-                if (!__all_sync(0xffffffffu, wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyDeq))) {
-                    ok = false;
-                    break;
-                }
                 tmem_st32(lane_addr + C::kACol0 + s * 32, v);
                 tmem_wait_st();
                 tc_fence_before();
@@ -452,7 +453,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
         tc_fence_after();
         constexpr int HALF = BN / 2;                  // columns per warp of a lane quarter
         const int cbeg = h * HALF;
-        if (have) {
+        if (have && y_tma) {
+            // bf16 tile [BN tokens][128 channels] in the (now idle) stage buffers,
+            // stored below by one TMA: every warp store writes 64 contiguous bytes
+            __nv_bfloat16 *ysm = (__nv_bfloat16 *)smem;
+            constexpr int CH = HALF < 64 ? HALF : 64;
+            for (int c = 0; c < HALF; c += CH) {
+                float acc[CH];
+                if (CH >= 32) {
+#pragma unroll
+                    for (int u = 0; u < CH / 32; ++u) tmem_ld32(lane_addr + cbeg + c + 32 * u, acc + 32 * u);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < CH / 8; ++u) tmem_ld8(lane_addr + cbeg + c + 8 * u, acc + 8 * u);
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < CH; ++j) ysm[(cbeg + c + j) * 128 + r] = __float2bfloat16_rn(acc[j]);
+            }
+        } else if (have) {
             // columns in chunks of CH (64, or the whole half when it is smaller),
             // all loads of a chunk issued before one wait
             constexpr int CH = HALF < 64 ? HALF : 64;
@@ -474,6 +493,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, int M, int N, int K, 
                         else partial[((size_t)split * M + m) * N + n] = acc[j];
                     }
                 }
+            }
+        }
+        if (y_tma) {
+            // make the tile visible to the TMA unit, then one thread stores it
+            // (rows past M and channels past N are clipped) and waits until
+            // shared memory has been read
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (threadIdx.x == 64 && *abort_flag == 0) {
+                asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                                 &tmap_y),
+                             "r"(smem_u32(smem)), "r"(n0), "r"(m0)
+                             : "memory");
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             }
         }
         if (splits > 1) {
@@ -571,7 +605,8 @@ TcPlan plan_tc(int64_t M, int64_t N, int64_t K)
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap &map, const TcPlan &p, int M, int N, int K, int glog2, int asym,
+cudaError_t launch_bn(const CUtensorMap &map, const CUtensorMap &qmap, const CUtensorMap &ymap, int y_tma,
+                      const TcPlan &p, int M, int N, int K, int glog2, int asym,
                       const uint32_t *qweight, const void *scales, const uint32_t *qzeros, void *Y, void *ws,
                       cudaStream_t stream)
 {
@@ -594,7 +629,7 @@ cudaError_t launch_bn(const CUtensorMap &map, const TcPlan &p, int M, int N, int
     }
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
     gemm_tc_kernel<BN><<<grid, kThreads, smem, stream>>>(
-        map, M, N, K, glog2, asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
+        map, qmap, ymap, y_tma, M, N, K, glog2, asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
         (__nv_bfloat16 *)Y, partial, counters, p.splits, p.kb_per_split);
     return cudaGetLastError();
 }
@@ -631,14 +666,37 @@ cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const
                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // the codes as 32-bit words [N][K/8]; one box = 128 channels x one 64-wide k-block
+    CUtensorMap qmap;
+    const cuuint64_t qdim[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+    const cuuint64_t qstride[1] = {(cuuint64_t)K / 2};
+    const cuuint32_t qbox[2] = {8u, 128u};
+    if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(qweight), qdim, qstride, qbox, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    // Y tiles leave through one TMA store per CTA when Y's rows are 16-byte
+    // aligned; otherwise (and for split-K partials) the epilogue stores directly
+    CUtensorMap ymap = map;
+    int y_tma = 0;
+    if (p.splits == 1 && ((uintptr_t)Y % 16) == 0 && (N * 2) % 16 == 0) {
+        const cuuint64_t ydim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        const cuuint64_t ystride[1] = {(cuuint64_t)N * 2};
+        const cuuint32_t ybox[2] = {128u, (cuuint32_t)p.BN};
+        if (enc(&ymap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, ydim, ystride, ybox, estride,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        y_tma = 1;
+    }
     const int glog2 = group == 32 ? 5 : group == 64 ? 6 : 7;
     const int asym = mode == W4_ASYM;
     switch (p.BN) {
-    case 16: return launch_bn<16>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    case 32: return launch_bn<32>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    case 64: return launch_bn<64>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    case 128: return launch_bn<128>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    default: return launch_bn<256>(map, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 16: return launch_bn<16>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 32: return launch_bn<32>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 64: return launch_bn<64>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 128: return launch_bn<128>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    default: return launch_bn<256>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
     }
 }
 
