@@ -210,10 +210,12 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v)
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
+// a + b on bf16 pairs.  The dequantization adds -(128 + zp), negated once per
+// group, because a subtraction of bf16 pairs costs an extra sign flip.
+__device__ __forceinline__ uint32_t bf2_add(uint32_t a, uint32_t b)
 {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -232,7 +234,7 @@ __device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c)
 }
 
 // Dequantization constants of one (channel, group): s_hi = bf16_rne(s16),
-// s_lo = s16 - s_hi (exact, <= 3 significant bits), Z = 128 + zp, each
+// s_lo = s16 - s_hi (exact, <= 3 significant bits), -Z = -(128 + zp), each
 // duplicated into both halves of a bf16x2.
 struct GroupConst {
     uint32_t shi, slo, z;
@@ -247,17 +249,20 @@ __device__ __forceinline__ GroupConst group_const(unsigned short s16bits, uint32
     GroupConst gc;
     gc.shi = h | (h << 16);
     gc.slo = l | (l << 16);
-    gc.z = 0x43004300u | (zp << 16) | zp;
+    gc.z = 0xC300C300u | (zp << 16) | zp;   // -(128 + zp)
     return gc;
 }
 
 // w^ for the adjacent elements (8c+2j, 8c+2j+1) held by packed word q:
 // (128+u) - (128+zp) is exact, D*s_lo is exact, and fma(D, s_hi, D*s_lo)
 // rounds the exact product D*s16 once to bf16.
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupConst &gc)
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const GroupConst &gc, uint32_t magic)
 {
-    const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
-    const uint32_t D = bf2_sub(v, gc.z);
+    // 128 + u: (q >> 4j) & 0x000F000F | magic in one LOP3, with magic =
+    // 0x43004300 held in a register (as an immediate it costs a second LOP3)
+    uint32_t v;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(q >> (4 * j)), "r"(0x000F000Fu), "r"(magic));
+    const uint32_t D = bf2_add(v, gc.z);
     return bf2_fma(D, gc.shi, bf2_mul(D, gc.slo));
 }
 
@@ -390,6 +395,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 
         // the codes arrive with the activations (TMA, full_b); only the scales
         // and zero-points are loaded here, D k-blocks of this warp ahead
+        uint32_t magic;                              // 0x43004300, opaque to the compiler
+        asm volatile("mov.b32 %0, 0x43004300;" : "=r"(magic));
         constexpr int D = 4;
         SlotData buf[D];
         auto fetch = [&](int i, SlotData &sd) {
@@ -437,8 +444,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 for (int w = 0; w < 4; ++w)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        v[4 * w + j] = dequant_pair(wa[w], j, c0);
-                        v[16 + 4 * w + j] = dequant_pair(wb[w], j, c1);
+                        v[4 * w + j] = dequant_pair(wa[w], j, c0, magic);
+                        v[16 + 4 * w + j] = dequant_pair(wb[w], j, c1, magic);
                     }
                 tmem_st32(lane_addr + C::kACol0 + s * 32, v);
                 tmem_wait_st();

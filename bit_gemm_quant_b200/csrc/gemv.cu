@@ -25,7 +25,8 @@
 //   * per k-box, each lane turns one (channel, group) scale and zero-point into
 //     the bf16x2 constants below and parks them in the warp's shared-memory
 //     slot, where the lanes that need them read them back (the scales and
-//     zero-points of the next box are loaded while this one is computed);
+//     zero-points of the next box are loaded while this one is computed, and
+//     the tile's whole scale and zero-point rows are asked into L2 at launch);
 //   * lane (g, t) = (lane/4, lane%4) reads, for channels g and g+8, the 16-byte
 //     chunks t and t+4 of the box (the swizzle makes these reads free of bank
 //     conflicts) and the activations of the same k from global memory;
@@ -95,10 +96,12 @@ __device__ __noinline__ bool wait_box(uint32_t bar, uint32_t parity)
     return true;
 }
 
-__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
+// a + b on bf16 pairs.  The dequantization adds -(128 + zp), negated once per
+// group, because a subtraction of bf16 pairs costs an extra sign flip.
+__device__ __forceinline__ uint32_t bf2_add(uint32_t a, uint32_t b)
 {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -127,26 +130,30 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 }
 
 // Per-(channel, group) dequantization constants, each duplicated into both
-// halves of a bf16x2: s_hi = bf16_rne(s16), s_lo = s16 - s_hi, Z = 128 + zp.
+// halves of a bf16x2: s_hi = bf16_rne(s16), s_lo = s16 - s_hi, and -Z = -(128 + zp).
 __device__ __forceinline__ uint4 group_const(unsigned short s16bits, uint32_t zp)
 {
     const float sf = __half2float(__ushort_as_half(s16bits));
     const __nv_bfloat16 hi = __float2bfloat16_rn(sf);
     const __nv_bfloat16 lo = __float2bfloat16_rn(sf - __bfloat162float(hi));   // exact
     const uint32_t h = __bfloat16_as_ushort(hi), l = __bfloat16_as_ushort(lo);
-    return make_uint4(h | (h << 16), l | (l << 16), 0x43004300u | (zp << 16) | zp, 0u);
+    return make_uint4(h | (h << 16), l | (l << 16), 0xC300C300u | (zp << 16) | zp, 0x43004300u);
 }
 
 // w^ for elements (2j, 2j+1) of packed word q.
 __device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const uint4 &gc)
 {
-    const uint32_t v = ((q >> (4 * j)) & 0x000F000Fu) | 0x43004300u;   // 128 + u, as bf16x2
-    const uint32_t D = bf2_sub(v, gc.z);
+    // 128 + u as bf16x2: (q >> 4j) & 0x000F000F | 0x43004300 in one LOP3; the
+    // constant 0x43004300 comes from shared memory (gc.w) so that it stays in a
+    // register instead of costing a second LOP3 per pair
+    uint32_t v;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(q >> (4 * j)), "r"(0x000F000Fu), "r"(gc.w));
+    const uint32_t D = bf2_add(v, gc.z);
     return bf2_fma(D, gc.x, bf2_mul(D, gc.y));
 }
 
 template <int G, int MODE, int MT>
-__global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 6 : 4)
+__global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 5 : 4)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
             __nv_bfloat16 *__restrict__ Y, int *err)
@@ -188,6 +195,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
     };
     if (lane == 0)
         for (int i = 0; i < kStages && i < nbw; ++i) issue(i);
+    if (threadIdx.x == 32) {                     // the tile's scales and zero-points, HBM -> L2
+        const int rows = min(16, N - r0);
+        prefetch_l2(scales + (size_t)r0 * NG, (size_t)rows * NG * 2);
+        if (MODE == W4_ASYM) prefetch_l2(qzeros + (size_t)r0 * ZW, (size_t)rows * ZW * 4);
+    }
 
     // scales / zero-points of the constants this lane computes for box i
     unsigned short sv[CPL];
