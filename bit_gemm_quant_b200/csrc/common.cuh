@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "w4.h"
 
 namespace w4 {
@@ -24,6 +26,35 @@ __device__ __forceinline__ void prefetch_l2(const void *p, size_t bytes)
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
         a += n;
     }
+}
+
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialization, so it may start while the previous kernel
+// of the stream drains; it runs only set-up that touches no global memory (its
+// shared-memory barriers, tensor-memory allocation, descriptor prefetch) before
+// pdl_wait(), which returns once the previous kernel has completed and its
+// writes are visible.  pdl_launch_dependents() then lets the next kernel start
+// its own set-up.  A previous kernel that does not trigger releases the next
+// one when it exits, so ordering against any other work on the stream is the
+// same as without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }

@@ -342,6 +342,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();                                                       // the previous kernel's writes are visible
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer --
@@ -635,10 +637,9 @@ cudaError_t launch_bn(const CUtensorMap &map, const CUtensorMap &qmap, const CUt
         counters = (unsigned *)((uint8_t *)ws + ((part + 255) & ~(size_t)255));
     }
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    gemm_tc_kernel<BN><<<grid, kThreads, smem, stream>>>(
-        map, qmap, ymap, y_tma, M, N, K, glog2, asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros,
-        (__nv_bfloat16 *)Y, partial, counters, p.splits, p.kb_per_split);
-    return cudaGetLastError();
+    return launch_pdl(gemm_tc_kernel<BN>, grid, dim3(kThreads), smem, stream, map, qmap, ymap, y_tma, M, N, K, glog2,
+                      asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros, (__nv_bfloat16 *)Y,
+                      partial, counters, p.splits, p.kb_per_split);
 }
 
 }  // namespace

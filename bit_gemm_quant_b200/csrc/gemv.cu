@@ -181,6 +181,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_q) : "memory");
     }
     __syncwarp();
+    pdl_wait();                                  // the previous kernel's writes are visible
+    pdl_launch_dependents();
     auto issue = [&](int i) {                    // lane 0: box i of this warp into stage i % kStages
         const int s = i % kStages;
         const int b = warp + kWarps * i;
@@ -343,10 +345,9 @@ cudaError_t launch_g(const CUtensorMap &map, const void *X, int64_t M, int64_t N
                      const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
 {
     const int64_t blocks = (N + 15) / 16;       // one 16-channel tile per CTA
-    gemv_kernel<G, MODE, MT><<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
-        map, (const uint4 *)X, (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros,
-        (__nv_bfloat16 *)Y, err);
-    return cudaGetLastError();
+    return launch_pdl(gemv_kernel<G, MODE, MT>, dim3((unsigned)blocks), dim3(kWarps * 32), 0, stream, map,
+                      (const uint4 *)X, (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros,
+                      (__nv_bfloat16 *)Y, err);
 }
 
 template <int MT>

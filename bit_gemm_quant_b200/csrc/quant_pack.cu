@@ -175,6 +175,8 @@ quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float
     const int64_t KC = K >> 5;                  // 32-weight chunks per row
     const int64_t NG = K / G;                   // groups per row
     const int64_t ZW = (NG + 7) >> 3;           // zero-point words per row
+    pdl_wait();                                 // the previous kernel's writes are visible
+    pdl_launch_dependents();
 
     // The work is the row-major sequence of 1024-weight items (32 chunks of a
     // row; the last item of a row may be shorter).  Warp w takes items w,
@@ -368,12 +370,12 @@ cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, u
     const int64_t cap = (int64_t)kNumSMs * per_sm;   // one resident wave; warps stride over rows
     if (blocks > cap) blocks = cap;
     if (s)
-        quant_pack_kernel<G, MODE, true><<<(unsigned)blocks, threads, 0, stream>>>(
-            (const uint4 *)W, N, K, (const float4 *)s, (uint4 *)qweight, (unsigned short *)scales, qzeros);
-    else
-        quant_pack_kernel<G, MODE, false><<<(unsigned)blocks, threads, 0, stream>>>(
-            (const uint4 *)W, N, K, nullptr, (uint4 *)qweight, (unsigned short *)scales, qzeros);
-    return cudaGetLastError();
+        return launch_pdl(quant_pack_kernel<G, MODE, true>, dim3((unsigned)blocks), dim3(threads), 0, stream,
+                          (const uint4 *)W, N, K, (const float4 *)s, (uint4 *)qweight, (unsigned short *)scales,
+                          qzeros);
+    return launch_pdl(quant_pack_kernel<G, MODE, false>, dim3((unsigned)blocks), dim3(threads), 0, stream,
+                      (const uint4 *)W, N, K, (const float4 *)nullptr, (uint4 *)qweight, (unsigned short *)scales,
+                      qzeros);
 }
 
 }  // namespace
