@@ -58,9 +58,12 @@ namespace w4 {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr int kStages = 4;                       // k-boxes in flight per warp
-constexpr int kBoxK = 256;                       // k per box: 32 words of 8 codes
+constexpr int kBoxK = 256;                       // k per TMA box: 32 words of 8 codes
 constexpr int kBoxBytes = 16 * 128;              // 16 channels x 128 bytes
+constexpr int kBoxesPerStage = 2;                // a pipeline stage is two boxes: 512 k
+constexpr int kStageK = kBoxK * kBoxesPerStage;
+constexpr int kStageBytes = kBoxBytes * kBoxesPerStage;
+constexpr int kStages = 2;                       // stages in flight per warp (8 KB)
 constexpr uint64_t kWaitLimitNs = 200000000ull;  // 200 ms; a box lands in microseconds
 constexpr int kErrGemvWait = 0x201, kErrGemvDrain = 0x202;
 
@@ -152,24 +155,38 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const uint4 
     return bf2_fma(D, gc.x, bf2_mul(D, gc.y));
 }
 
+// Dynamic shared-memory layout of one GEMV CTA.
+template <int G, int MT>
+struct GemvSmem {
+    static constexpr int kConstOff = kWarps * kStages * kStageBytes;
+    static constexpr int kRedOff = kConstOff + kWarps * 16 * (kStageK / G) * 16;
+    static constexpr int kBarOff = kRedOff + kWarps * 32 * 4 * MT * 4;
+    static constexpr int kBytes = kBarOff + kWarps * kStages * 8 + 1024;   // + alignment slack
+};
+
 template <int G, int MODE, int MT>
 __global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 5 : 4)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
             __nv_bfloat16 *__restrict__ Y, int *err)
 {
-    constexpr int GPB = kBoxK / G;               // groups per box and channel
-    constexpr int CPL = 16 * GPB / 32;           // constants computed per lane and box
-    __shared__ __align__(1024) uint8_t sbox[kWarps][kStages][kBoxBytes];
-    __shared__ uint4 sconst[kWarps][16 * GPB];
-    __shared__ float red[kWarps][32][4 * MT];
-    __shared__ __align__(8) uint64_t full[kWarps][kStages];
+    constexpr int GPB = kStageK / G;             // groups per stage and channel
+    constexpr int CPL = 16 * GPB / 32;           // constants computed per lane and stage
+    // dynamic shared memory: the stages (1024-byte aligned for the swizzle),
+    // the constants, the cross-warp reduction and the barriers
+    extern __shared__ uint8_t smem_raw[];
+    using L = GemvSmem<G, MT>;
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    auto sbox = (uint8_t(*)[kStages][kStageBytes])(smem);
+    auto sconst = (uint4(*)[16 * GPB])(smem + L::kConstOff);
+    auto red = (float(*)[32][4 * MT])(smem + L::kRedOff);
+    auto full = (uint64_t(*)[kStages])(smem + L::kBarOff);
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int NG = K / G, ZW = (NG + 7) >> 3;
-    const int NB = (K + kBoxK - 1) / kBoxK;      // k-boxes per channel
-    const int nbw = (NB - warp + kWarps - 1) / kWarps;   // boxes of this warp: warp, warp+4, ...
+    const int NS = (K + kStageK - 1) / kStageK;  // stages per channel
+    const int nsw = (NS - warp + kWarps - 1) / kWarps;   // stages of this warp: warp, warp+4, ...
     const int r0 = (int)blockIdx.x * 16;
 
     const uint32_t bar0 = smem_u32(&full[warp][0]);
@@ -183,41 +200,43 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
     __syncwarp();
     pdl_wait();                                  // the previous kernel's writes are visible
     pdl_launch_dependents();
-    auto issue = [&](int i) {                    // lane 0: box i of this warp into stage i % kStages
+    auto issue = [&](int i) {                    // lane 0: stage i of this warp into slot i % kStages
         const int s = i % kStages;
-        const int b = warp + kWarps * i;
+        const int sb = warp + kWarps * i;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar0 + 8 * s),
-                     "r"(kBoxBytes)
+                     "r"(kStageBytes)
                      : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-            "[%2];" ::"r"(box0 + s * kBoxBytes),
-            "l"(&tmap_q), "r"(bar0 + 8 * s), "r"(b * 32), "r"(r0)
-            : "memory");
+#pragma unroll
+        for (int bb = 0; bb < kBoxesPerStage; ++bb)   // a box past the end of K is zero-filled
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+                "[%2];" ::"r"(box0 + s * kStageBytes + bb * kBoxBytes),
+                "l"(&tmap_q), "r"(bar0 + 8 * s), "r"((sb * kBoxesPerStage + bb) * 32), "r"(r0)
+                : "memory");
     };
     if (lane == 0)
-        for (int i = 0; i < kStages && i < nbw; ++i) issue(i);
+        for (int i = 0; i < kStages && i < nsw; ++i) issue(i);
     if (threadIdx.x == 32) {                     // the tile's scales and zero-points, HBM -> L2
         const int rows = min(16, N - r0);
         prefetch_l2(scales + (size_t)r0 * NG, (size_t)rows * NG * 2);
         if (MODE == W4_ASYM) prefetch_l2(qzeros + (size_t)r0 * ZW, (size_t)rows * ZW * 4);
     }
 
-    // scales / zero-points of the constants this lane computes for box i
+    // scales / zero-points of the constants this lane computes for stage i
     unsigned short sv[CPL];
     uint32_t zv[CPL];
     auto load_consts = [&](int i) {
-        const int b = warp + kWarps * i;
+        const int sb = warp + kWarps * i;
 #pragma unroll
         for (int u = 0; u < CPL; ++u) {
-            const int idx = lane + 32 * u, row = r0 + (idx & 15), j = b * GPB + (idx >> 4);
+            const int idx = lane + 32 * u, row = r0 + (idx & 15), j = sb * GPB + (idx >> 4);
             const bool ok = row < N && j < NG;
             sv[u] = ok ? __ldg(scales + (size_t)row * NG + j) : (unsigned short)0;
             if (MODE == W4_ASYM) zv[u] = ok ? (__ldg(qzeros + (size_t)row * ZW + (j >> 3)) >> (4 * (j & 7))) & 0xFu : 0u;
             else zv[u] = 8u;
         }
     };
-    if (nbw > 0) load_consts(0);
+    if (nsw > 0) load_consts(0);
 
     // two accumulator sets (the first and the second MMA of every word pair)
     // halve the dependent chain of MMAs
@@ -226,56 +245,50 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][e] = acc2[mt][e] = 0.f;
+    // a token past M reads token M-1: its MMA column is never stored
+    const uint4 *xrows[MT];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) xrows[mt] = X + (size_t)min(g + 8 * mt, M - 1) * (K / 8);
 
     bool ok = true;
     int i = 0;
-    for (; i < nbw; ++i) {
-        const int b = warp + kWarps * i;
+    for (; i < nsw; ++i) {
+        const int sb = warp + kWarps * i;
         const int s = i % kStages;
-        // constants of this box into the warp's slot, then the next box's loads
-        __syncwarp();                            // every lane is done with the previous box's slot
+        // constants of this stage into the warp's slot, then the next stage's loads
+        __syncwarp();                            // every lane is done with the previous stage's slot
 #pragma unroll
         for (int u = 0; u < CPL; ++u) sconst[warp][lane + 32 * u] = group_const(sv[u], zv[u]);
-        if (i + 1 < nbw) load_consts(i + 1);
+        if (i + 1 < nsw) load_consts(i + 1);
         __syncwarp();
         if (!wait_box(bar0 + 8 * s, (uint32_t)(i / kStages) & 1u)) {
             ok = false;
             break;
         }
-        // this lane's codes: channels g and g+8, chunks t and t+4 (128-byte swizzle)
-        const uint8_t *bx = &sbox[warp][s][0];
-        const uint4 qa0 = *(const uint4 *)(bx + g * 128 + ((t ^ g) << 4));
-        const uint4 qa1 = *(const uint4 *)(bx + g * 128 + (((t + 4) ^ g) << 4));
-        const uint4 qb0 = *(const uint4 *)(bx + (g + 8) * 128 + ((t ^ g) << 4));
-        const uint4 qb1 = *(const uint4 *)(bx + (g + 8) * 128 + (((t + 4) ^ g) << 4));
-        __syncwarp();                            // the stage is read: refill it
-        if (lane == 0 && i + kStages < nbw) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue(i + kStages);
-        }
+        const uint8_t *st = &sbox[warp][s][0];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = t + 4 * h;             // chunk of this half
+        for (int h = 0; h < 2 * kBoxesPerStage; ++h) {
+            const int bb = h >> 1;               // box of this chunk
+            const int c = t + 4 * (h & 1);       // chunk of the box (16 bytes of a 128-byte row)
+            // this lane's codes: channels g and g+8, chunk c (128-byte swizzle)
+            const uint4 wa4 = *(const uint4 *)(st + bb * kBoxBytes + g * 128 + ((c ^ g) << 4));
+            const uint4 wb4 = *(const uint4 *)(st + bb * kBoxBytes + (g + 8) * 128 + ((c ^ g) << 4));
             // first k of the chunk; a chunk past the end of K (K is a multiple of
             // 32, chunks are whole) reads the last chunk's activations instead:
             // its codes are zero-filled by TMA and its groups' constants have
             // s16 = 0, so every w^ there is 0 and the activations only need to
             // be finite
-            const int k0 = min(b * kBoxK + c * 32, K - 32);
-            const uint4 ca = sconst[warp][(g) + 16 * ((c * 32) / G)];
-            const uint4 cb = sconst[warp][(g + 8) + 16 * ((c * 32) / G)];
-            const uint4 wa4 = h ? qa1 : qa0, wb4 = h ? qb1 : qb0;
+            const int k0 = min(sb * kStageK + bb * kBoxK + c * 32, K - 32);
+            const int gl = (bb * kBoxK + c * 32) / G;     // group of the chunk within the stage
+            const uint4 ca = sconst[warp][g + 16 * gl];
+            const uint4 cb = sconst[warp][(g + 8) + 16 * gl];
             const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
             const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
             uint4 xv[MT][4];
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                // a token past M reads token M-1: its MMA column is never stored
-                const int tok = min(g + 8 * mt, M - 1);
-                const uint4 *xrow = X + ((size_t)tok * K + k0) / 8;
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int w = 0; w < 4; ++w) xv[mt][w] = __ldg(xrow + w);
-            }
+                for (int w = 0; w < 4; ++w) xv[mt][w] = __ldg(xrows[mt] + k0 / 8 + w);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const uint32_t a0 = dequant_pair(wa[w], 0, ca), a1 = dequant_pair(wa[w], 1, ca);
@@ -289,13 +302,18 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
                 }
             }
         }
+        __syncwarp();                            // the stage is read: refill it
+        if (lane == 0 && i + kStages < nsw) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(i + kStages);
+        }
     }
     if (!ok) {
         // a box never landed: record it, wait (bounded) for the copies this warp
         // still has in flight, and leave the tile unwritten
         if (lane == 0) {
             atomicCAS(err, 0, kErrGemvWait);
-            for (int j = i; j < nbw && j < i + kStages; ++j)
+            for (int j = i; j < nsw && j < i + kStages; ++j)
                 if (!wait_box(bar0 + 8 * (j % kStages), (uint32_t)(j / kStages) & 1u)) atomicCAS(err, 0, kErrGemvDrain);
         }
     }
@@ -345,7 +363,15 @@ cudaError_t launch_g(const CUtensorMap &map, const void *X, int64_t M, int64_t N
                      const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
 {
     const int64_t blocks = (N + 15) / 16;       // one 16-channel tile per CTA
-    return launch_pdl(gemv_kernel<G, MODE, MT>, dim3((unsigned)blocks), dim3(kWarps * 32), 0, stream, map,
+    constexpr int smem = GemvSmem<G, MT>::kBytes;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(gemv_kernel<G, MODE, MT>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    return launch_pdl(gemv_kernel<G, MODE, MT>, dim3((unsigned)blocks), dim3(kWarps * 32), smem, stream, map,
                       (const uint4 *)X, (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros,
                       (__nv_bfloat16 *)Y, err);
 }
