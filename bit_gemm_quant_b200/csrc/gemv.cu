@@ -15,9 +15,10 @@
 // the dequantization costs about 2.5 issue slots per weight, which is close to
 // the issue budget of the SMs at HBM speed, so the kernel must stream the codes
 // without spending instructions on it):
-//   * a CTA (4 warps) owns a tile of 16 output channels and all of K; warp w
-//     takes the 256-wide k-boxes w, w+4, w+8, ... and the four partial tiles
-//     are summed in shared memory at the end (no global scratch);
+//   * a CTA (4 warps, or 8 when there are fewer than two tiles per SM) owns a
+//     tile of 16 output channels and all of K; warp w takes the 512-wide
+//     k-stages w, w+W, w+2W, ... and the partial tiles are summed in shared
+//     memory at the end (no global scratch);
 //   * the codes stream HBM -> shared memory by TMA (one 2-D box of 16 rows x
 //     128 bytes per k-box, 128-byte swizzle), four boxes in flight per warp on
 //     the warp's own mbarrier ring, so a resident CTA keeps 32 KB of reads
@@ -57,7 +58,6 @@
 namespace w4 {
 namespace {
 
-constexpr int kWarps = 4;
 constexpr int kBoxK = 256;                       // k per TMA box: 32 words of 8 codes
 constexpr int kBoxBytes = 16 * 128;              // 16 channels x 128 bytes
 constexpr int kBoxesPerStage = 2;                // a pipeline stage is two boxes: 512 k
@@ -156,7 +156,7 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t q, int j, const uint4 
 }
 
 // Dynamic shared-memory layout of one GEMV CTA.
-template <int G, int MT>
+template <int G, int MT, int kWarps>
 struct GemvSmem {
     static constexpr int kConstOff = kWarps * kStages * kStageBytes;
     static constexpr int kRedOff = kConstOff + kWarps * 16 * (kStageK / G) * 16;
@@ -164,8 +164,8 @@ struct GemvSmem {
     static constexpr int kBytes = kBarOff + kWarps * kStages * 8 + 1024;   // + alignment slack
 };
 
-template <int G, int MODE, int MT>
-__global__ void __launch_bounds__(kWarps * 32, MT == 1 ? 5 : 4)
+template <int G, int MODE, int MT, int kWarps>
+__global__ void __launch_bounds__(kWarps * 32, kWarps == 8 ? 2 : (MT == 1 ? 5 : 4))
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
             __nv_bfloat16 *__restrict__ Y, int *err)
@@ -175,7 +175,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const uint4 *__restrict_
     // dynamic shared memory: the stages (1024-byte aligned for the swizzle),
     // the constants, the cross-warp reduction and the barriers
     extern __shared__ uint8_t smem_raw[];
-    using L = GemvSmem<G, MT>;
+    using L = GemvSmem<G, MT, kWarps>;
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     auto sbox = (uint8_t(*)[kStages][kStageBytes])(smem);
     auto sconst = (uint4(*)[16 * GPB])(smem + L::kConstOff);
@@ -358,22 +358,33 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-template <int G, int MODE, int MT>
-cudaError_t launch_g(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
-                     const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
+template <int G, int MODE, int MT, int W>
+cudaError_t launch_gw(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
+                      const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
 {
     const int64_t blocks = (N + 15) / 16;       // one 16-channel tile per CTA
-    constexpr int smem = GemvSmem<G, MT>::kBytes;
+    constexpr int smem = GemvSmem<G, MT, W>::kBytes;
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(gemv_kernel<G, MODE, MT>,
+        const cudaError_t e = cudaFuncSetAttribute(gemv_kernel<G, MODE, MT, W>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_pdl(gemv_kernel<G, MODE, MT>, dim3((unsigned)blocks), dim3(kWarps * 32), smem, stream, map,
+    return launch_pdl(gemv_kernel<G, MODE, MT, W>, dim3((unsigned)blocks), dim3(W * 32), smem, stream, map,
                       (const uint4 *)X, (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros,
                       (__nv_bfloat16 *)Y, err);
+}
+
+// Few tiles (fewer than two per SM) get 8 warps each, so that the SMs still
+// hold enough warps to hide latency; otherwise 4 warps per tile.
+template <int G, int MODE, int MT>
+cudaError_t launch_g(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
+                     const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
+{
+    if ((N + 15) / 16 <= 2 * kNumSMs)
+        return launch_gw<G, MODE, MT, 8>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    return launch_gw<G, MODE, MT, 4>(map, X, M, N, K, scales, qzeros, Y, err, stream);
 }
 
 template <int MT>
