@@ -62,7 +62,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["w4", "reference"], default="w4")
-    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "awq"], default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -628,11 +628,119 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------------ awq search --
+
+AWQ_SHAPE = dict(M=128, N=4096, K=4096, group=128, mode=1, n_alpha=20)
+
+
+def awq_bytes(M, N, K, group, mode, n_alpha):
+    """Algorithmic bytes of one search: per alpha a folded quantization and a
+    W4A16 product (plus X/s), once the reference product W X^T."""
+    per_alpha = (roofline.quant_pack_bytes(N, K, group, mode, True) + roofline.gemm_bytes(M, N, K, group, mode)
+                 + 4 * M * K + 6 * M * N)
+    return n_alpha * per_alpha + 2 * M * K + 2 * N * K + 4 * M * N
+
+
+def run_awq(args, rank, world, local_rank):
+    """The AWQ scale search (page 2, AWQ section) over a decode-sized layer and
+    128 calibration rows with 1% outlier input channels; one step is one whole
+    search (20 alphas)."""
+    import torch
+    import bit_gemm_quant_b200 as w4
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    w4.lib()
+    pk = roofline.peaks(ROOT)
+    sh = AWQ_SHAPE
+    M, N, K, g, mode, na = sh["M"], sh["N"], sh["K"], sh["group"], sh["mode"], sh["n_alpha"]
+    W = torch.from_numpy(synth.weights(21 + 1000 * rank, N, K, 0.02, 0.01, 5.0).view(np.int16)).to(device)
+    X = torch.from_numpy(synth.activations(22 + 1000 * rank, M, K, 0.01, 20.0).view(np.int16)).to(device)
+    W, X = W.view(torch.bfloat16), X.view(torch.bfloat16)
+    need = w4.w4_awq_workspace_bytes(M, N, K, g, mode)
+    ws = torch.empty(need, dtype=torch.uint8, device=device)
+    losses = torch.empty(na, dtype=torch.float64, device=device)
+    best = torch.empty(1, dtype=torch.int32, device=device)
+    s_best = torch.empty(K, dtype=torch.float32, device=device)
+
+    def step():
+        st = w4.w4_awq_search(w4._ptr(W), w4._ptr(X), N, K, M, g, mode, na, w4._ptr(losses), w4._ptr(best),
+                              w4._ptr(s_best), w4._ptr(ws), need, w4._stream_handle(None))
+        if st != w4.W4_OK:
+            raise w4.W4Error(st, "w4_awq_search")
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    K_steps = args.steps
+    graph = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(device)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cs):
+        for _ in range(K_steps):
+            step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(smi_gpu_id(local_rank))
+    sampler.start()
+    sampler.mark_begin()
+    t_end = time.time() + 1.5
+    while time.time() < t_end:
+        graph.replay()
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    e1.synchronize()
+    barrier()
+    local_ms = e0.elapsed_time(e1)
+    sampler.mark_end()
+    clocks = sampler.stop()
+    del graph
+    work = K_steps * awq_bytes(M, N, K, g, mode, na)
+    max_ms, total = aggregate(local_ms, work, device)
+    value = total / (max_ms * 1e-3) / 1e9
+    per_search_s = max_ms * 1e-3 / K_steps
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K_steps,
+            "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / K_steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "AWQ scale search: W[%d,%d] bf16, X[%d,%d] calibration rows with 1%% outlier "
+                                   "channels x20, asymmetric INT4 g=%d, %d alphas; step = one whole search"
+                                   % (N, K, M, K, g, na),
+                       "timing": "K searches captured in one CUDA graph, replayed between CUDA events after 1.5 s "
+                                 "of untimed replays; max over ranks",
+                       "parallelism": "replicas (dp%d), no data-path collective" % world},
+            "roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(value / world / pk["hbm_gbs"], 4), "traffic": None,
+                         "kernel": "w4_awq_search (whole search)",
+                         "algorithmic_per_launch": awq_bytes(M, N, K, g, mode, na)},
+            "searches_per_s": round(world / per_search_s, 2),
+            "best_alpha_index": int(best.cpu().numpy()[0]),
+            "cpu_baseline": None, "e2e": None,
+            "gpu_launches": K_steps * (2 + na * 5 + 2) * world, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return 0
+    if args.workload == "awq":
+        run_awq(args, rank, world, local_rank)
         return 0
     run_w4(args, rank, world, local_rank)
     return 0

@@ -42,6 +42,10 @@ def lib() -> ctypes.CDLL:
         L.w4a16_gemm.restype = I
         L.w4a16_gemm_noalloc.argtypes = [P, I64, I64, I64, P, P, P, I, I, P, P]
         L.w4a16_gemm_noalloc.restype = I
+        L.w4_awq_workspace_bytes.argtypes = [I64, I64, I64, I, I]
+        L.w4_awq_workspace_bytes.restype = SZ
+        L.w4_awq_search.argtypes = [P, P, I64, I64, I64, I, I, I, P, P, P, P, SZ, P]
+        L.w4_awq_search.restype = I
         L.w4_status_string.argtypes = [I]
         L.w4_status_string.restype = ctypes.c_char_p
         L.w4_layout_version.argtypes = []
@@ -69,6 +73,16 @@ def w4a16_gemm(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace, w
 
 def w4a16_gemm_noalloc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, stream) -> int:
     return lib().w4a16_gemm_noalloc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, stream)
+
+
+def w4_awq_workspace_bytes(M, N, K, group, mode) -> int:
+    return int(lib().w4_awq_workspace_bytes(M, N, K, group, mode))
+
+
+def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, workspace, workspace_bytes,
+                  stream) -> int:
+    return lib().w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, workspace,
+                               workspace_bytes, stream)
 
 
 def w4_status_string(status: int) -> str:
@@ -156,3 +170,21 @@ def gemm_noalloc(X, qweight, scales, qzeros, group: int, mode: int, N: int | Non
     if st != W4_OK:
         raise W4Error(st, "w4a16_gemm_noalloc")
     return Y
+
+
+def awq_search(W, X, group: int = 128, mode: int = SYM, n_alpha: int = 20, stream=None):
+    """AWQ scale search over bf16 CUDA tensors W[N,K] and calibration X[M,K].
+    Returns (losses fp64 [n_alpha], best index tensor, s_best fp32 [K])."""
+    import torch
+    N, K = W.shape
+    M = X.shape[0]
+    need = w4_awq_workspace_bytes(M, N, K, group, mode)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    losses = torch.empty(n_alpha, dtype=torch.float64, device=W.device)
+    best = torch.empty(1, dtype=torch.int32, device=W.device)
+    s_best = torch.empty(K, dtype=torch.float32, device=W.device)
+    st = w4_awq_search(_ptr(W), _ptr(X), N, K, M, group, mode, n_alpha, _ptr(losses), _ptr(best), _ptr(s_best),
+                       _ptr(ws), ws.numel(), _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_awq_search")
+    return losses, best, s_best

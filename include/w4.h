@@ -127,6 +127,38 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
                      void *workspace, size_t workspace_bytes, w4_stream_t stream);
 
 /*
+ * w4_awq_workspace_bytes -- device scratch that w4_awq_search needs (0 for
+ * malformed arguments).
+ */
+size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode);
+
+/*
+ * w4_awq_search -- the AWQ smoothing-scale search (page 2, AWQ section, the
+ * awq_search_scale listing: a grid search over alpha for the per-input-channel
+ * scale s that minimises the error of the quantized layer on calibration data).
+ *   W        bf16 [N][K] weight, 32-byte aligned.
+ *   X        bf16 [M][K] calibration activations, 16-byte aligned; every input
+ *            channel must have a nonzero mean magnitude.
+ *   group, mode: as for w4_quant_pack.
+ *   n_alpha  grid size, 2..4096: alpha_i = i / (n_alpha - 1) in fp64.
+ *   losses   out, fp64 [n_alpha] device array (8-byte aligned).
+ *   best     out, int device scalar: the first index of the smallest loss.
+ *   s_best   out, fp32 [K] device array (16-byte aligned): s for that alpha,
+ *            ready to pass to w4_quant_pack (and to divide X by upstream).
+ *   workspace / workspace_bytes: w4_awq_workspace_bytes(M, N, K, group, mode)
+ *            bytes, 256-byte aligned, contents need not be initialised.
+ * For each alpha: act[k] = mean_m |x[m][k]| (fp64); s = act^alpha /
+ * mean_k act^alpha in fp64, rounded once to fp32; Q = w4_quant_pack(W, s);
+ * Y_q = w4a16_gemm(bf16(X / s), Q) (the product (W^ / s) X^T as the W4A16
+ * path computes it); loss = mean over all M x N outputs of
+ * (Y_ref - Y_q)^2 in fp64, with Y_ref = X W^T accumulated in fp32.
+ * Asynchronous on `stream`; errors as for the other entry points.
+ */
+w4_status w4_awq_search(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
+                        int n_alpha, double *losses, int *best, float *s_best, void *workspace,
+                        size_t workspace_bytes, w4_stream_t stream);
+
+/*
  * w4a16_gemm_noalloc -- w4a16_gemm for callers that cannot allocate device
  * memory (a stream capture that must not allocate, a host whose allocator
  * owns all device memory, a plug-in that only receives its input and output
