@@ -72,6 +72,33 @@ def test_gemv_edge_sizes(w4, N, K):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K", [(1, 4800, 8192), (7, 1000, 2304), (12, 37904, 256)])
+def test_gemv_more_shapes(w4, M, N, K):
+    """Long rows (K = 8192), a ragged K (2304 = 9 k-boxes) and many one-box rows
+    (K = 256, N = 37904 channels: 2369 tiles, more than one resident wave)."""
+    W = synth.weights(N + K + M, N, K, 0.02, 0.01, 5.0)
+    X = synth.activations(N + K + M, M, K, 0.01, 40.0)
+    check(gpu_path(w4, W, X, 128, ASYM), W, X, 128, ASYM)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M", [1, 12])
+def test_gemv_is_deterministic(w4, M):
+    """Repeated calls give the same bits."""
+    import torch
+    N, K = 4096, 4096
+    W = synth.weights(93 + M, N, K, 0.02)
+    X = synth.activations(93 + M, M, K, 0.01, 40.0)
+    q, sc, z = w4.quant_pack(dev_bf16(W), 128, ASYM)
+    Xd = dev_bf16(X)
+    Ys = [host_bf16_as_f64(w4.gemm(Xd, q, sc, z, 128, ASYM)) for _ in range(5)]
+    torch.cuda.synchronize()
+    assert all(np.array_equal(Ys[0], Y) for Y in Ys[1:])
+    check(Ys[0], W, X, 128, ASYM)
+    assert w4.w4_device_error() == 0
+
+
+@pytest.mark.gpu
 def test_tiny_workload(w4):
     (p,) = synth.workload("tiny")
     W, X = p.W(), p.X()
