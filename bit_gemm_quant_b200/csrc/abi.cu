@@ -40,6 +40,7 @@ w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode
     if (!W || !qweight || !scales) return W4_ERR_INVALID_ARG;
     if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
     if (N < 1 || K < 8 || K % group != 0 || !fits(N, K)) return W4_ERR_INVALID_ARG;
+    if (N > INT32_MAX - 65536 || K > INT32_MAX - 65536) return W4_ERR_UNSUPPORTED;   // 32-bit row / column indices
     if ((mode == W4_ASYM) != (qzeros != nullptr)) return W4_ERR_INVALID_ARG;
     if (!aligned(W, 32) || !aligned(qweight, 16) || !aligned(scales, 2)) return W4_ERR_INVALID_ARG;
     if (s && !aligned(s, 16)) return W4_ERR_INVALID_ARG;

@@ -9,36 +9,43 @@
 //
 // Design (HBM-bound stream: 2 B read + about 0.5 B written per weight; the
 // SMs' issue budget at full bandwidth is about 11 instructions per weight, so
-// the per-weight work is kept to a handful of instructions):
-//   * one resident wave of CTAs; the matrix is a row-major sequence of
-//     1024-weight items and warp w takes items w, w + nwarps, ..., so the
-//     warps' shares differ by at most one item; a warp loads its next item
-//     before it processes the current one and asks L2 for the one after
-//     (cp.async.bulk.prefetch); a lane owns 32 consecutive weights, which
-//     always lie in one group (g = 32, 64, 128 is 1, 2 or 4 lanes), read with
-//     two 32-byte loads;
+// the per-weight work is kept to a handful of instructions and the per-group
+// work is spread over as many weights as registers allow):
+//   * one resident wave of CTAs; the matrix is a row-major sequence of items
+//     of 32 lane slices of 64 consecutive weights (2048 weights), and warp w
+//     takes items w, w + nwarps, ..., so the warps' shares differ by at most
+//     one item; a warp asks L2 for its item two steps ahead
+//     (cp.async.bulk.prefetch) and reads its slice with four 32-byte loads; a
+//     slice lies in one group (g = 64), in two (g = 32), or in half of one
+//     (g = 128: two lanes);
 //   * group amax / min / max: packed bf16x2 min and max over the lane's raw
-//     words (fp32 comparisons after the fold) and at most two
-//     __shfl_xor_sync steps; the per-group IEEE divisions (scale and zero
-//     point) and the reciprocal are amortized over 32 weights per lane;
+//     words (fp32 comparisons after the fold) and at most one
+//     __shfl_xor_sync; the per-group IEEE divisions (scale and zero point)
+//     and the reciprocal are amortized over 64 weights per lane;
+//   * with a fold, the 64 weights are folded once per item (w' = fl32(w * s))
+//     and kept as fp32 pairs; the smoothing vector is staged once per CTA in
+//     shared memory, each 64-factor slice rotated by (slice % 8) float4 so
+//     that the lanes' reads of their slices (256 bytes apart) do not collide
+//     on banks, and the weights are read past L1 so that it keeps s;
 //   * per weight the code is rint(w'/s16) with IEEE semantics.  The fast path
 //     adds the magic constant 1.5*2^23 + zp to w' * rcp(s16), which leaves
 //     0x4B400000 + u in the float's bits, and computes the exact residual
 //     rho = w' - r * s16 (Sterbenz: r * s16 has <= 16 significant bits), two
-//     weights per fma/add instruction.  A pair whose |rho| reaches s16/2 -- an
-//     exact tie of the quotient (common with bf16 weights) or a rounding the
-//     approximation got wrong -- is flagged and recomputed exactly from the
-//     raw words parked in shared memory (ties to even); groups whose fp16
-//     scale saturated or is subnormal take an IEEE-division path;
+//     weights per fma/add instruction.  A packed word (8 weights) whose
+//     largest |rho| reaches s16/2 -- an exact tie of the quotient (common
+//     with bf16 weights) or a rounding the approximation got wrong -- is
+//     flagged and recomputed exactly from its raw weights, read again from
+//     cache (ties to even); groups whose fp16 scale saturated or is subnormal
+//     take an IEEE-division path;
 //   * y is monotonic in w', so the asymmetric clamp to [0, 15] (needed before
 //     packing: a code of -1 or 16 would borrow from or carry into the next
 //     nibble) runs only in warps where some group's extremes map outside;
 //   * packing: with bits(y) = C + u (C's low byte 0), one IMAD y_b*16 + y_a
 //     puts the byte u_a | u_b << 4 in the low byte; three PRMTs assemble the
-//     word (even elements in the low half-word), and each lane stores its 4
-//     words as one 16-byte store (a warp writes 512 contiguous bytes);
-//   * zero-points of 8 groups are OR-reduced with __shfl_xor_sync inside their
-//     8*g/32-lane segment and stored once per word.
+//     word (even elements in the low half-word), and each lane stores its 8
+//     words as two 16-byte stores;
+//   * zero-points of 8 groups are OR-reduced with __shfl_xor_sync across the
+//     4, 8 or 16 lanes that hold them and stored once per word.
 #include "common.cuh"
 
 namespace w4 {
@@ -57,11 +64,19 @@ __device__ __forceinline__ float rcp_approx(float d)
     return r;
 }
 
+// 32 bytes of weights.  With STREAM the load does not allocate in L1 (the
+// folded path keeps its smoothing factors there instead).
+template <bool STREAM>
 __device__ __forceinline__ void ld32(const uint4 *p, uint32_t (&v)[8])
 {
-    asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
-                 : "l"(p));
+    if (STREAM)
+        asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                     : "l"(p));
+    else
+        asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                     : "l"(p));
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
@@ -106,40 +121,50 @@ __device__ __forceinline__ float2 weight_pair(uint32_t v, float2 sp)
     return FOLD ? __fmul2_rn(w, sp) : w;
 }
 
-// Fast-path codes of the lane's 32 weights: y = fl(w' * rcp(s16) + magic)
-// holds r + zp (or r + 8) in its low bits, r = rint of the approximate
-// quotient; rho = w' - r * s16 is exact.  Bit p of the returned flags marks the
-// weight pair p if either residual reaches half a step (|rho| >= s16 / 2):
-// exact ties of the quotient and roundings the approximation got wrong.  With
-// CLAMP the asymmetric codes are clamped to [0, 15] before packing (a code of
-// -1 or 16 would borrow from or carry into the neighbouring nibble); without
-// it the caller has shown that every y lies in range.  The arithmetic runs on
-// pairs (fma / add of two fp32 lanes per instruction, each correctly rounded).
+// Per-group parameters of the fast path.
+struct QParams {
+    float inv, magic, d, hd, ymax;
+    int zp;
+};
+
+// Fast-path codes of one 32-weight chunk (16 raw words): y = fl(w' * rcp(s16)
+// + magic) holds r + zp (or r + 8) in its low bits, r = rint of the
+// approximate quotient; rho = w' - r * s16 is exact.  Bit w of the returned
+// flags marks packed word w (8 weights) if any of its residuals reaches half a
+// step (|rho| >= s16 / 2): exact ties of the quotient and roundings the
+// approximation got wrong.  With CLAMP the asymmetric codes are clamped to
+// [0, 15] before packing (a code of -1 or 16 would borrow from or carry into
+// the neighbouring nibble); without it the caller has shown that every y lies
+// in range.  The arithmetic runs on pairs (fma / add of two fp32 lanes per
+// instruction, each correctly rounded).  With FOLD, xf holds the chunk's 16
+// folded weight pairs (w * s in fp32) and cur is not read.
 template <int MODE, bool FOLD, bool CLAMP>
-__device__ __forceinline__ uint32_t encode(const uint32_t (&cur)[16], const float2 (&sp)[16], float inv,
-                                           float magic, float d, float hd, float ymax, uint32_t (&wd)[4])
+__device__ __forceinline__ uint32_t encode(const uint32_t *cur, const float2 *xf, const QParams &q,
+                                           uint32_t (&wd)[4])
 {
-    const float2 inv2 = make_float2(inv, inv), mg2 = make_float2(magic, magic);
-    const float2 nmg2 = make_float2(-magic, -magic), nd2 = make_float2(-d, -d);
+    const float2 inv2 = make_float2(q.inv, q.inv), mg2 = make_float2(q.magic, q.magic);
+    const float2 nmg2 = make_float2(-q.magic, -q.magic), nd2 = make_float2(-q.d, -q.d);
     uint32_t flags = 0u;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
         uint32_t yb[8];
+        float m = 0.f;                           // largest |rho| of the word
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int p = 4 * w + j;
-            const float2 x = weight_pair<FOLD>(cur[p], sp[p]);
+            const float2 x = FOLD ? xf[p] : weight_pair<false>(cur[p], make_float2(1.f, 1.f));
             float2 y = __ffma2_rn(x, inv2, mg2);
             if (MODE == W4_ASYM && CLAMP) {
-                y.x = fmaxf(fminf(y.x, ymax), kMagic);
-                y.y = fmaxf(fminf(y.y, ymax), kMagic);
+                y.x = fmaxf(fminf(y.x, q.ymax), kMagic);
+                y.y = fmaxf(fminf(y.y, q.ymax), kMagic);
             }
             const float2 r = __fadd2_rn(y, nmg2);
             const float2 rho = __ffma2_rn(r, nd2, x);
-            if (fmaxf(fabsf(rho.x), fabsf(rho.y)) >= hd) flags |= 1u << p;
+            m = fmaxf(m, fmaxf(fabsf(rho.x), fabsf(rho.y)));
             yb[2 * j] = __float_as_uint(y.x);
             yb[2 * j + 1] = __float_as_uint(y.y);
         }
+        if (m >= q.hd) flags |= 1u << w;
         wd[w] = pack_word(yb);
     }
     return flags;
@@ -148,211 +173,292 @@ __device__ __forceinline__ uint32_t encode(const uint32_t (&cur)[16], const floa
 // The exact code of one weight (its fast-path y recomputed, then the tie or
 // the wrong rounding resolved from the exact residual).
 template <int MODE>
-__device__ __forceinline__ uint32_t exact_code(float x, float inv, float magic, float d, float hd, float ymax, int zp)
+__device__ __forceinline__ uint32_t exact_code(float x, const QParams &q)
 {
-    float y = __fmaf_rn(x, inv, magic);
-    if (MODE == W4_ASYM) y = fmaxf(fminf(y, ymax), kMagic);
-    const float r = __fsub_rn(y, magic);
-    const float rho = __fmaf_rn(-r, d, x);
+    float y = __fmaf_rn(x, q.inv, q.magic);
+    if (MODE == W4_ASYM) y = fmaxf(fminf(y, q.ymax), kMagic);
+    const float r = __fsub_rn(y, q.magic);
+    const float rho = __fmaf_rn(-r, q.d, x);
     const float ar = fabsf(rho);
     // beyond half a step, or an exact tie with r odd: one step toward rho
-    const int odd = (int)(__float_as_uint(y) ^ (uint32_t)zp) & 1;
-    int q = (int)r;
-    if (ar > hd || (ar == hd && odd)) q += (rho > 0.f) ? 1 : -1;
-    return (MODE == W4_SYM) ? (uint32_t)(min(max(q, -8), 7) + 8) : (uint32_t)min(max(q + zp, 0), 15);
+    const int odd = (int)(__float_as_uint(y) ^ (uint32_t)q.zp) & 1;
+    int c = (int)r;
+    if (ar > q.hd || (ar == q.hd && odd)) c += (rho > 0.f) ? 1 : -1;
+    return (MODE == W4_SYM) ? (uint32_t)(min(max(c, -8), 7) + 8) : (uint32_t)min(max(c + q.zp, 0), 15);
+}
+
+// The code of one weight by IEEE division (groups whose fp16 scale saturated
+// or is subnormal).
+template <int MODE>
+__device__ __forceinline__ uint32_t division_code(float x, const QParams &q)
+{
+    const float c = rintf(__fdiv_rn(x, q.d));
+    return (MODE == W4_SYM) ? (uint32_t)((int)fminf(fmaxf(c, -8.f), 7.f) + 8)
+                            : (uint32_t)(int)fminf(fmaxf(c + (float)q.zp, 0.f), 15.f);
+}
+
+// Scale, zero-point and fast-path parameters of a group from the extremes mn
+// <= 0 <= mx (asymmetric) or the largest magnitude a (symmetric) of its w'.
+template <int MODE>
+__device__ __forceinline__ QParams group_params(float a, float mn, float mx, unsigned short &s16, bool &exact_only)
+{
+    QParams q;
+    float s32, hi = 0.f;
+    if (MODE == W4_SYM) s32 = __fdiv_rn(a, 7.0f);
+    else s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
+    q.d = __half2float(__ushort_as_half(s16));
+    if (MODE == W4_SYM) {
+        q.zp = 8;
+    } else {
+        q.zp = (q.d > 0.f) ? (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, q.d)), 0.f), 15.f) : 0;
+        hi = (float)(15 - q.zp);
+    }
+    // the fast path assumes a normal, unsaturated fp16 scale (or a zero one)
+    exact_only = (s16 == 0x7BFF) || (q.d > 0.f && q.d < 6.103515625e-05f);
+    q.inv = (q.d > 0.f) ? rcp_approx(q.d) : 0.f;
+    q.magic = kMagic + (float)q.zp;              // exact: 1.5*2^23 + zp < 2^24
+    q.hd = (q.d > 0.f) ? 0.5f * q.d : __int_as_float(0x7F800000);
+    q.ymax = q.magic + hi;
+    return q;
 }
 
 template <int G, int MODE, bool FOLD>
-__global__ void __launch_bounds__(256, 3)
-quant_pack_kernel(const uint4 *__restrict__ W, int64_t N, int64_t K, const float4 *__restrict__ s,
+__global__ void __launch_bounds__(256, 2)
+quant_pack_kernel(const uint32_t *__restrict__ W, int N, int K, const float *__restrict__ s, int s_staged,
                   uint4 *__restrict__ qweight, unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros)
 {
-    constexpr int LPG = G / 32;                 // lanes per group
-    __shared__ uint4 stash[4][256];             // raw words, [quarter][thread]: for the rare exact fix
+    constexpr int GPL = (G == 32) ? 2 : 1;       // groups per lane: a lane owns 64 consecutive weights
+    constexpr int LPG = (G == 128) ? 2 : 1;      // lanes per group
     const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t KC = K >> 5;                  // 32-weight chunks per row
-    const int64_t NG = K / G;                   // groups per row
-    const int64_t ZW = (NG + 7) >> 3;           // zero-point words per row
-    pdl_wait();                                 // the previous kernel's writes are visible
+    const int warp0 = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+    const int KW = K >> 1;                       // raw words (bf16 pairs) per row
+    const int KP = (K + 63) >> 6;                // 64-weight slices per row (the last may hold 32)
+    const int NG = K / G, ZW = (NG + 7) >> 3;
+    pdl_wait();                                  // the previous kernel's writes are visible
     pdl_launch_dependents();
 
-    // The work is the row-major sequence of 1024-weight items (32 chunks of a
-    // row; the last item of a row may be shorter).  Warp w takes items w,
-    // w + nwarps, w + 2 nwarps, ... (so every warp gets the same number of
-    // items, whatever N and K), loads its next item before it processes the
-    // current one and asks L2 for the item after that.  Lanes past the end of
-    // a row keep zero words (they are not stored).
-    const int64_t IPR = (KC + 31) >> 5;         // items per row
-    const int64_t step_rows = nwarps / IPR, step_items = nwarps % IPR;
-    auto advance = [&](int64_t &row, int64_t &item) {
+    // With a fold and s_staged, the smoothing vector is staged in shared memory
+    // once per block: slice c (64 factors, 16 float4) is rotated by c % 8
+    // float4, so that the 32 lanes' reads of "their" float4 i hit 8 different
+    // 16-byte bank groups (the slices are 256 bytes apart).
+    extern __shared__ float4 s_sm[];
+    if (FOLD && s_staged) {
+        const int n4 = K >> 2, n4p = 16 * ((K + 63) >> 6);   // a half slice at the end is padded with 0
+        for (int j = threadIdx.x; j < n4p; j += blockDim.x) {
+            const int c = j >> 4, pos = j & 15;
+            s_sm[16 * c + ((pos + (c & 7)) & 15)] = j < n4 ? __ldg((const float4 *)s + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+    }
+
+    // The work is the row-major sequence of items of 32 slices (2048 weights;
+    // the last item of a row may be shorter).  Warp w takes items w,
+    // w + nwarps, ... (so every warp gets the same number of items, whatever N
+    // and K are) and asks L2 for its items two steps ahead.
+    const int IPR = (KP + 31) >> 5;              // items per row
+    const int step_rows = nwarps / IPR, step_items = nwarps % IPR;
+    auto advance = [&](int &row, int &item) {
         row += step_rows;
         item += step_items;
-        if (item >= IPR) { item -= IPR; ++row; }
+        if (item >= IPR) {
+            item -= IPR;
+            ++row;
+        }
     };
-    int64_t n = warp0 / IPR, it = warp0 % IPR;  // row and item-in-row of the current item
-    uint32_t cur[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    if (n < N && 32 * it + lane < KC) {
-        const uint4 *p = W + n * (K >> 3) + 4 * (32 * it + lane);
-        ld32(p, *(uint32_t(*)[8])&cur[0]);
-        ld32(p + 2, *(uint32_t(*)[8])&cur[8]);
+    auto prefetch_item = [&](int row, int item) {  // lane 0: one item, HBM -> L2
+        if (row < N) {
+            const int w0 = 1024 * item;
+            prefetch_l2(W + (size_t)row * KW + w0, (size_t)min(1024, KW - w0) * 4);
+        }
+    };
+    int n = warp0 / IPR, it = warp0 % IPR;       // row and item-in-row of the current item
+    int pn = n, pit = it;                        // the item two steps ahead
+    advance(pn, pit);
+    if (lane == 0) {
+        prefetch_item(n, it);
+        prefetch_item(pn, pit);
     }
-    while (n < N) {
-        const int64_t c0 = 32 * it;             // first chunk of the current item
-        int64_t nn = n, nit = it;
-        advance(nn, nit);
-        uint32_t nxt[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (nn < N && 32 * nit + lane < KC) {
-            const uint4 *p = W + nn * (K >> 3) + 4 * (32 * nit + lane);
-            ld32(p, *(uint32_t(*)[8])&nxt[0]);
-            ld32(p + 2, *(uint32_t(*)[8])&nxt[8]);
-        }
-        if (lane == 0) {                        // the item after next, HBM -> L2
-            int64_t pn = nn, pit = nit;
-            advance(pn, pit);
-            if (pn < N) {
-                const int64_t pc = 32 * pit, nch = (KC - pc) < 32 ? (KC - pc) : 32;
-                prefetch_l2(W + pn * (K >> 3) + 4 * pc, (size_t)nch * 64);
-            }
-        }
-        {
-            const int64_t c = c0 + lane;        // this lane's chunk
-            const bool valid = c < KC;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                stash[q][threadIdx.x] = make_uint4(cur[4 * q], cur[4 * q + 1], cur[4 * q + 2], cur[4 * q + 3]);
-            float2 sp[16];                      // smoothing factors of the weight pairs
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 f = (FOLD && valid) ? __ldg(s + 8 * c + i) : make_float4(1.f, 1.f, 1.f, 1.f);
-                sp[2 * i] = make_float2(f.x, f.y);
-                sp[2 * i + 1] = make_float2(f.z, f.w);
-            }
+    advance(pn, pit);
 
-            // ---- group statistics, scale and zero-point ----
-            float lmin, lmax;                   // extremes of this lane's 32 weights w'
-            if (!FOLD) {                        // on the raw bf16 pairs: one min and one max per pair
-                uint32_t pmin = cur[0], pmax = cur[0];
+    while (n < N) {
+        if (lane == 0) prefetch_item(pn, pit);
+        advance(pn, pit);
+        const int cp = 32 * it + lane;           // this lane's slice
+        const bool valid = cp < KP;
+        const int cpl = valid ? cp : KP - 1;     // a lane past the row end reads the last slice (not stored)
+        const bool valid1 = 64 * cpl + 32 < K;   // the slice's second 32-weight chunk is in the row
+        const uint32_t *src = W + (size_t)n * KW + 32 * cpl;
+        uint32_t cur[32];
+        ld32<FOLD>((const uint4 *)src, *(uint32_t(*)[8]) & cur[0]);
+        ld32<FOLD>((const uint4 *)(src + 8), *(uint32_t(*)[8]) & cur[8]);
+        if (valid1) {
+            ld32<FOLD>((const uint4 *)(src + 16), *(uint32_t(*)[8]) & cur[16]);
+            ld32<FOLD>((const uint4 *)(src + 24), *(uint32_t(*)[8]) & cur[24]);
+        } else {
 #pragma unroll
-                for (int i = 1; i < 16; ++i) { pmin = bmin2(pmin, cur[i]); pmax = bmax2(pmax, cur[i]); }
+            for (int i = 16; i < 32; ++i) cur[i] = 0u;
+        }
+        // with a smoothing fold: the 64 weights w' = fl32(w * s), once per item
+        float2 xf[FOLD ? 32 : 1];
+        if (FOLD) {
+            const float4 *sv = (const float4 *)(s + 64 * (size_t)cpl);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float4 f = make_float4(0.f, 0.f, 0.f, 0.f);   // (the missing half of a half slice)
+                if (s_staged) f = s_sm[16 * cpl + ((i + (cpl & 7)) & 15)];
+                else if (i < 8 || valid1) f = __ldg(sv + i);
+                xf[2 * i] = weight_pair<true>(cur[2 * i], make_float2(f.x, f.y));
+                xf[2 * i + 1] = weight_pair<true>(cur[2 * i + 1], make_float2(f.z, f.w));
+            }
+        }
+
+        // ---- group statistics, scales and zero-points ----
+        QParams qp[GPL];
+        unsigned short s16[GPL];
+        bool exact_only = false, clamp = false;
+#pragma unroll
+        for (int gi = 0; gi < GPL; ++gi) {
+            constexpr int WPG = 32 / GPL;        // raw words of the group held by this lane
+            float lmin, lmax;                    // extremes of this lane's part of the group (w')
+            if (!FOLD) {                         // on the raw bf16 pairs: one min and one max per pair
+                uint32_t pmin = cur[WPG * gi], pmax = cur[WPG * gi];
+#pragma unroll
+                for (int i = 1; i < WPG; ++i) {
+                    pmin = bmin2(pmin, cur[WPG * gi + i]);
+                    pmax = bmax2(pmax, cur[WPG * gi + i]);
+                }
                 lmin = fminf(bf16lo_to_f32(pmin), bf16hi_to_f32(pmin));
                 lmax = fmaxf(bf16lo_to_f32(pmax), bf16hi_to_f32(pmax));
             } else {
                 lmin = lmax = 0.f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 x = weight_pair<true>(cur[i], sp[i]);
+                for (int i = 0; i < WPG; ++i) {
+                    const float2 x = xf[(WPG * gi + i) % (FOLD ? 32 : 1)];
                     lmin = fminf(lmin, fminf(x.x, x.y));
                     lmax = fmaxf(lmax, fmaxf(x.x, x.y));
                 }
             }
-            float d, mn = 0.f, mx = 0.f, hi = 0.f;
-            int zp;
-            unsigned short s16;
+            float a = 0.f, mn = 0.f, mx = 0.f;
             if (MODE == W4_SYM) {
-                float a = fmaxf(fabsf(lmin), fabsf(lmax));
-#pragma unroll
-                for (int off = LPG / 2; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-                const float s32 = __fdiv_rn(a, 7.0f);
-                s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
-                d = __half2float(__ushort_as_half(s16));
-                zp = 8;
+                a = fmaxf(fabsf(lmin), fabsf(lmax));
+                if (LPG == 2) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
             } else {
                 mn = fminf(0.f, lmin);
                 mx = fmaxf(0.f, lmax);
-#pragma unroll
-                for (int off = LPG / 2; off > 0; off >>= 1) {
-                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                if (LPG == 2) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 }
-                const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-                s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
-                d = __half2float(__ushort_as_half(s16));
-                zp = (d > 0.f) ? (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, d)), 0.f), 15.f) : 0;
-                hi = (float)(15 - zp);
             }
-            // the fast path assumes a normal, unsaturated fp16 scale (or a zero one)
-            const bool exact_only = (s16 == 0x7BFF) || (d > 0.f && d < 6.103515625e-05f);
-            const float inv = (d > 0.f) ? rcp_approx(d) : 0.f;
-            const float magic = kMagic + (float)zp;   // exact: 1.5*2^23 + zp < 2^24
-            const float hd = (d > 0.f) ? 0.5f * d : __int_as_float(0x7F800000);
-            const float ymax = magic + hi;
-
-            // ---- codes ----
-            // y is monotonic in w', so when the group's extremes mn and mx map into
-            // [0, 15] every weight of the group does and no clamp is needed; the
-            // (rare) warps with a group whose extremes fall outside run the clamped
-            // variant.  Symmetric codes never leave [1, 15]: |w'/s16| <= 7 (1 + 2^-11).
-            uint32_t wd[4], flags;
-            bool clamp = false;
+            bool eo;
+            qp[gi] = group_params<MODE>(a, mn, mx, s16[gi], eo);
+            exact_only |= eo;
+            // y is monotonic in w', so when the group's extremes map into [0, 15]
+            // every weight of the group does and no clamp is needed; symmetric
+            // codes never leave [1, 15]: |w'/s16| <= 7 (1 + 2^-11)
             if (MODE == W4_ASYM)
-                clamp = __fmaf_rn(mn, inv, magic) < kMagic || __fmaf_rn(mx, inv, magic) > ymax;
-            if (MODE == W4_ASYM && __any_sync(0xffffffffu, clamp))
-                flags = encode<MODE, FOLD, true>(cur, sp, inv, magic, d, hd, ymax, wd);
-            else
-                flags = encode<MODE, FOLD, false>(cur, sp, inv, magic, d, hd, ymax, wd);
-            if (__any_sync(0xffffffffu, flags != 0u)) {
-                // fix the flagged pairs from the raw words parked in shared memory
-                // (a warp has one in about two items with bf16 weights: exact ties
-                // are common when the fp16 scale has few significant bits)
-                uint32_t m = flags;
-                while (m) {
-                    const int p = __ffs(m) - 1;
-                    m &= m - 1u;
-                    const uint32_t v = ((const uint32_t *)&stash[p >> 2][threadIdx.x])[p & 3];
-                    float2 sv = make_float2(1.f, 1.f);
-                    if (FOLD) sv = __ldg((const float2 *)s + 16 * c + p);
-                    const float2 x = weight_pair<FOLD>(v, sv);
-                    const uint32_t u0 = exact_code<MODE>(x.x, inv, magic, d, hd, ymax, zp);
-                    const uint32_t u1 = exact_code<MODE>(x.y, inv, magic, d, hd, ymax, zp);
-                    // elements 2p, 2p+1: nibble (p & 3) of the low and of the high half-word
-                    const int sh = 4 * (p & 3), w = p >> 2;
-                    const uint32_t keep = ~((0xFu << sh) | (0xFu << (16 + sh)));
-                    const uint32_t val = (u0 << sh) | (u1 << (16 + sh));
-                    wd[0] = (w == 0) ? ((wd[0] & keep) | val) : wd[0];
-                    wd[1] = (w == 1) ? ((wd[1] & keep) | val) : wd[1];
-                    wd[2] = (w == 2) ? ((wd[2] & keep) | val) : wd[2];
-                    wd[3] = (w == 3) ? ((wd[3] & keep) | val) : wd[3];
-                }
-            }
-            uint4 out = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-            if (exact_only) {                   // saturated or subnormal scale: IEEE division
-                uint32_t wx[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-                for (int p = 0; p < 16; ++p) {
-                    const float2 x = weight_pair<FOLD>(cur[p], sp[p]);
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float q = rintf(__fdiv_rn(h ? x.y : x.x, d));
-                        int u;
-                        if (MODE == W4_SYM) u = (int)fminf(fmaxf(q, -8.f), 7.f) + 8;
-                        else u = (int)fminf(fmaxf(q + (float)zp, 0.f), 15.f);
-                        wx[p >> 2] |= (uint32_t)u << nibble_shift(2 * (p & 3) + h);
-                    }
-                }
-                out = make_uint4(wx[0], wx[1], wx[2], wx[3]);
-            }
+                clamp |= __fmaf_rn(mn, qp[gi].inv, qp[gi].magic) < kMagic ||
+                         __fmaf_rn(mx, qp[gi].inv, qp[gi].magic) > qp[gi].ymax;
+        }
 
-            const int64_t j = (c * 32) / G;     // group of this lane
-            if (valid) {
-                qweight[n * KC + c] = out;      // 16 bytes = the 32 codes of this lane
-                if ((lane % LPG) == 0) scales[n * NG + j] = s16;
-            }
-            if (MODE == W4_ASYM) {
-                // OR the zero-points of 8 consecutive groups (8*LPG lanes) into one word
-                uint32_t z = (valid && (lane % LPG) == 0) ? ((uint32_t)zp << (4 * (int)(j & 7))) : 0u;
+        // ---- codes ----
+        uint32_t wa[4], wb[4], flags;
+        if (MODE == W4_ASYM && __any_sync(0xffffffffu, clamp))
+            flags = encode<MODE, FOLD, true>(cur, xf, qp[0], wa) |
+                    (encode<MODE, FOLD, true>(cur + 16, xf + (FOLD ? 16 : 0), qp[GPL - 1], wb) << 4);
+        else
+            flags = encode<MODE, FOLD, false>(cur, xf, qp[0], wa) |
+                    (encode<MODE, FOLD, false>(cur + 16, xf + (FOLD ? 16 : 0), qp[GPL - 1], wb) << 4);
+        if (__any_sync(0xffffffffu, flags != 0u)) {
+            // fix the flagged words from the raw weights (read again, from cache)
+            uint32_t m = flags;
+            while (m) {
+                const int w = __ffs(m) - 1;
+                m &= m - 1u;
+                const int c = w >> 2;            // chunk of the word
+                if (c == 1 && !valid1) continue;   // (a half slice's missing chunk is not stored)
+                QParams q = qp[0];
+                if (GPL == 2 && c == 1) q = qp[GPL - 1];
+                const uint4 raw = __ldg((const uint4 *)(src + 4 * w));
+                const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t word = 0u;
 #pragma unroll
-                for (int off = 1; off < 8 * LPG; off <<= 1) z |= __shfl_xor_sync(0xffffffffu, z, off);
-                if (valid && (lane % (8 * LPG)) == 0) qzeros[n * ZW + (j >> 3)] = z;
+                for (int e = 0; e < 4; ++e) {
+                    float2 sp = make_float2(1.f, 1.f);
+                    if (FOLD) {
+                        const float2 *s2 = (const float2 *)(s + 64 * (size_t)cpl) + 4 * w + e;
+                        sp = __ldg(s2);
+                    }
+                    const float2 x = weight_pair<FOLD>(rw[e], sp);
+                    word |= exact_code<MODE>(x.x, q) << nibble_shift(2 * e);
+                    word |= exact_code<MODE>(x.y, q) << nibble_shift(2 * e + 1);
+                }
+                wa[0] = (w == 0) ? word : wa[0];
+                wa[1] = (w == 1) ? word : wa[1];
+                wa[2] = (w == 2) ? word : wa[2];
+                wa[3] = (w == 3) ? word : wa[3];
+                wb[0] = (w == 4) ? word : wb[0];
+                wb[1] = (w == 5) ? word : wb[1];
+                wb[2] = (w == 6) ? word : wb[2];
+                wb[3] = (w == 7) ? word : wb[3];
             }
         }
+        if (exact_only) {                        // saturated or subnormal scale: IEEE division
 #pragma unroll
-        for (int i = 0; i < 16; ++i) cur[i] = nxt[i];
-        n = nn;
-        it = nit;
+            for (int w = 0; w < 8; ++w) {
+                QParams q = qp[0];
+                if (GPL == 2 && w >= 4) q = qp[GPL - 1];
+                uint32_t word = 0u;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = FOLD ? xf[(4 * w + e) % (FOLD ? 32 : 1)]
+                                          : weight_pair<false>(cur[4 * w + e], make_float2(1.f, 1.f));
+                    word |= division_code<MODE>(x.x, q) << nibble_shift(2 * e);
+                    word |= division_code<MODE>(x.y, q) << nibble_shift(2 * e + 1);
+                }
+                if (w < 4) wa[w] = word;
+                else wb[w - 4] = word;
+            }
+        }
+
+        // ---- stores: 2 x 16 bytes of codes, the scales, the zero-points ----
+        if (valid) {
+            uint4 *dst = qweight + (size_t)n * (K >> 5) + 2 * cp;
+            dst[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            if (valid1) dst[1] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+            unsigned short *srow = scales + (size_t)n * NG;
+            if (G == 32) {
+                srow[2 * cp] = s16[0];
+                if (valid1) srow[2 * cp + 1] = s16[GPL - 1];
+            } else if (G == 64) {
+                srow[cp] = s16[0];
+            } else if ((lane & 1) == 0) {
+                srow[cp >> 1] = s16[0];
+            }
+        }
+        if (MODE == W4_ASYM) {
+            // OR the zero-points of 8 consecutive groups into one word
+            uint32_t z = 0u;
+            if (G == 32) {
+                if (valid) z = ((uint32_t)qp[0].zp << (4 * ((2 * cp) & 7))) |
+                               (valid1 ? (uint32_t)qp[GPL - 1].zp << (4 * ((2 * cp + 1) & 7)) : 0u);
+            } else if (G == 64) {
+                if (valid) z = (uint32_t)qp[0].zp << (4 * (cp & 7));
+            } else {
+                if (valid && (lane & 1) == 0) z = (uint32_t)qp[0].zp << (4 * ((cp >> 1) & 7));
+            }
+            constexpr int LPW = (G == 32) ? 4 : (G == 64) ? 8 : 16;   // lanes per zero-point word
+#pragma unroll
+            for (int off = 1; off < LPW; off <<= 1) z |= __shfl_xor_sync(0xffffffffu, z, off);
+            if (valid && (lane & (LPW - 1)) == 0) qzeros[(size_t)n * ZW + cp / LPW] = z;
+        }
+        advance(n, it);
     }
 }
+
+constexpr int kMaxStagedS = 64 * 1024;          // bytes of smoothing factors staged in shared memory
 
 template <int G, int MODE>
 cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, uint32_t *qweight, void *scales,
@@ -365,17 +471,28 @@ cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, u
                                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_pack_kernel<G, MODE, false>, threads, 0);
         if (e != cudaSuccess || per_sm < 1) per_sm = 1;
     }
-    const int64_t items = N * ((K / 32 + 31) / 32);   // 1024-weight items
+    const int64_t items = N * ((K / 64 + 1 + 31) / 32);   // 2048-weight items (upper bound)
     int64_t blocks = (items + 7) / 8;            // one warp per item at most
     const int64_t cap = (int64_t)kNumSMs * per_sm;   // one resident wave; warps stride over rows
     if (blocks > cap) blocks = cap;
-    if (s)
-        return launch_pdl(quant_pack_kernel<G, MODE, true>, dim3((unsigned)blocks), dim3(threads), 0, stream,
-                          (const uint4 *)W, N, K, (const float4 *)s, (uint4 *)qweight, (unsigned short *)scales,
-                          qzeros);
+    if (s) {
+        // the smoothing vector in shared memory when it fits in 64 KB
+        static bool attr_set = false;
+        if (!attr_set) {
+            const cudaError_t e = cudaFuncSetAttribute(quant_pack_kernel<G, MODE, true>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxStagedS);
+            if (e != cudaSuccess) return e;
+            attr_set = true;
+        }
+        const size_t sbytes = (size_t)((K + 63) / 64) * 256;   // whole 64-factor slices
+        const int staged = (sbytes <= (size_t)kMaxStagedS) ? 1 : 0;
+        return launch_pdl(quant_pack_kernel<G, MODE, true>, dim3((unsigned)blocks), dim3(threads),
+                          staged ? sbytes : 0, stream, (const uint32_t *)W, (int)N, (int)K, s, staged,
+                          (uint4 *)qweight, (unsigned short *)scales, qzeros);
+    }
     return launch_pdl(quant_pack_kernel<G, MODE, false>, dim3((unsigned)blocks), dim3(threads), 0, stream,
-                      (const uint4 *)W, N, K, (const float4 *)nullptr, (uint4 *)qweight, (unsigned short *)scales,
-                      qzeros);
+                      (const uint32_t *)W, (int)N, (int)K, (const float *)nullptr, 0, (uint4 *)qweight,
+                      (unsigned short *)scales, qzeros);
 }
 
 }  // namespace
