@@ -660,7 +660,7 @@ def run_awq(args, rank, world, local_rank):
     W = torch.from_numpy(synth.weights(21 + 1000 * rank, N, K, 0.02, 0.01, 5.0).view(np.int16)).to(device)
     X = torch.from_numpy(synth.activations(22 + 1000 * rank, M, K, 0.01, 20.0).view(np.int16)).to(device)
     W, X = W.view(torch.bfloat16), X.view(torch.bfloat16)
-    need = w4.w4_awq_workspace_bytes(M, N, K, g, mode)
+    need = w4.w4_awq_workspace_bytes(M, N, K, g, mode, na)
     ws = torch.empty(need, dtype=torch.uint8, device=device)
     losses = torch.empty(na, dtype=torch.float64, device=device)
     best = torch.empty(1, dtype=torch.int32, device=device)
@@ -725,7 +725,7 @@ def run_awq(args, rank, world, local_rank):
             "searches_per_s": round(world / per_search_s, 2),
             "best_alpha_index": int(best.cpu().numpy()[0]),
             "cpu_baseline": None, "e2e": None,
-            "gpu_launches": K_steps * (2 + na * 5 + 2) * world, "clocks": clocks,
+            "gpu_launches": K_steps * (4 + na * 3 + 2) * world, "clocks": clocks,
         }
         print(json.dumps(out), flush=True)
     if world > 1:

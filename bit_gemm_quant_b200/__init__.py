@@ -42,7 +42,7 @@ def lib() -> ctypes.CDLL:
         L.w4a16_gemm.restype = I
         L.w4a16_gemm_noalloc.argtypes = [P, I64, I64, I64, P, P, P, I, I, P, P]
         L.w4a16_gemm_noalloc.restype = I
-        L.w4_awq_workspace_bytes.argtypes = [I64, I64, I64, I, I]
+        L.w4_awq_workspace_bytes.argtypes = [I64, I64, I64, I, I, I]
         L.w4_awq_workspace_bytes.restype = SZ
         L.w4_awq_search.argtypes = [P, P, I64, I64, I64, I, I, I, P, P, P, P, SZ, P]
         L.w4_awq_search.restype = I
@@ -75,8 +75,8 @@ def w4a16_gemm_noalloc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, stre
     return lib().w4a16_gemm_noalloc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, stream)
 
 
-def w4_awq_workspace_bytes(M, N, K, group, mode) -> int:
-    return int(lib().w4_awq_workspace_bytes(M, N, K, group, mode))
+def w4_awq_workspace_bytes(M, N, K, group, mode, n_alpha) -> int:
+    return int(lib().w4_awq_workspace_bytes(M, N, K, group, mode, n_alpha))
 
 
 def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, workspace, workspace_bytes,
@@ -178,7 +178,7 @@ def awq_search(W, X, group: int = 128, mode: int = SYM, n_alpha: int = 20, strea
     import torch
     N, K = W.shape
     M = X.shape[0]
-    need = w4_awq_workspace_bytes(M, N, K, group, mode)
+    need = w4_awq_workspace_bytes(M, N, K, group, mode, n_alpha)
     ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
     losses = torch.empty(n_alpha, dtype=torch.float64, device=W.device)
     best = torch.empty(1, dtype=torch.int32, device=W.device)

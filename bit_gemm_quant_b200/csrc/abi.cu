@@ -85,10 +85,11 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
-size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode)
+size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode, int n_alpha)
 {
     if (M < 1 || N < 1 || K < 1 || !group_ok(group) || !mode_ok(mode) || K % group != 0) return 0;
-    return w4::awq_workspace_bytes(M, N, K, group, mode);
+    if (n_alpha < 2 || n_alpha > 4096 || !fits(M, K) || !fits(M * K, n_alpha)) return 0;
+    return w4::awq_workspace_bytes(M, N, K, group, mode, n_alpha);
 }
 
 w4_status w4_awq_search(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
@@ -102,7 +103,8 @@ w4_status w4_awq_search(const void *W, const void *X, int64_t N, int64_t K, int6
     if (!aligned(W, 32) || !aligned(X, 16) || !aligned(losses, 8) || !aligned(best, 4) || !aligned(s_best, 16) ||
         !aligned(workspace, 256))
         return W4_ERR_INVALID_ARG;
-    if (workspace_bytes < w4::awq_workspace_bytes(M, N, K, group, mode)) return W4_ERR_INVALID_ARG;
+    if (!fits(M * K, n_alpha) || workspace_bytes < w4::awq_workspace_bytes(M, N, K, group, mode, n_alpha))
+        return W4_ERR_INVALID_ARG;
     if (M > INT32_MAX || N > INT32_MAX - 16 || K > INT32_MAX || M * K > INT32_MAX || M * N > INT32_MAX)
         return W4_ERR_UNSUPPORTED;
     const cudaError_t e = w4::launch_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best,

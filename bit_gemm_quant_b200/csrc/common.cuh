@@ -72,7 +72,7 @@ void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size
 cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                            const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
                            cudaStream_t stream);
-size_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode);
+size_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode, int n_alpha);
 cudaError_t launch_awq_search(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
                               int n_alpha, double *losses, int *best, float *s_best, void *ws, cudaStream_t stream);
 int read_and_clear_device_error();

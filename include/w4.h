@@ -127,10 +127,12 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
                      void *workspace, size_t workspace_bytes, w4_stream_t stream);
 
 /*
- * w4_awq_workspace_bytes -- device scratch that w4_awq_search needs (0 for
- * malformed arguments).
+ * w4_awq_workspace_bytes -- device scratch that w4_awq_search needs for a
+ * grid of n_alpha points (0 for malformed arguments).  It holds, among
+ * others, the scale vector of every alpha (n_alpha * K fp32) and X divided by
+ * each of them (n_alpha * M * K bf16).
  */
-size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode);
+size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode, int n_alpha);
 
 /*
  * w4_awq_search -- the AWQ smoothing-scale search (page 2, AWQ section, the
@@ -145,8 +147,8 @@ size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mo
  *   best     out, int device scalar: the first index of the smallest loss.
  *   s_best   out, fp32 [K] device array (16-byte aligned): s for that alpha,
  *            ready to pass to w4_quant_pack (and to divide X by upstream).
- *   workspace / workspace_bytes: w4_awq_workspace_bytes(M, N, K, group, mode)
- *            bytes, 256-byte aligned, contents need not be initialised.
+ *   workspace / workspace_bytes: w4_awq_workspace_bytes(M, N, K, group, mode,
+ *            n_alpha) bytes, 256-byte aligned, contents need not be initialised.
  * For each alpha: act[k] = mean_m |x[m][k]| (fp64); s = act^alpha /
  * mean_k act^alpha in fp64, rounded once to fp32; Q = w4_quant_pack(W, s);
  * Y_q = w4a16_gemm(bf16(X / s), Q) (the product (W^ / s) X^T as the W4A16

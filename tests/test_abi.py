@@ -110,3 +110,31 @@ def test_workspace_query_is_host_only(w4):
     for M in (1, 4, 8, 16, 32, 512, 8192):
         assert w4.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
     assert w4.w4a16_workspace_bytes(1, 4096, 4096, 128) == 0
+
+
+def test_awq_workspace_query_is_host_only(w4):
+    a = w4.w4_awq_workspace_bytes(128, 4096, 4096, 128, 1, 20)
+    b = w4.w4_awq_workspace_bytes(128, 4096, 4096, 128, 1, 40)
+    assert a > 0 and b > a                       # scale vectors and divided activations per alpha
+    assert b - a >= 20 * (4096 * 4 + 128 * 4096 * 2)
+    assert w4.w4_awq_workspace_bytes(128, 4096, 4096, 128, 1, 1) == 0    # a grid needs two points
+    assert w4.w4_awq_workspace_bytes(128, 4096, 4000, 128, 1, 20) == 0   # K not a multiple of g
+    assert w4.w4_awq_workspace_bytes(0, 4096, 4096, 128, 1, 20) == 0
+
+
+def test_awq_search_rejects_malformed_arguments_before_any_launch(w4):
+    P = 1 << 12                                  # never dereferenced: rejected first
+    ok = dict(W=P, X=P, N=256, K=512, M=8, g=128, mode=0, na=8, losses=P, best=P, s=P, ws=P, wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return w4.w4_awq_search(a["W"], a["X"], a["N"], a["K"], a["M"], a["g"], a["mode"], a["na"], a["losses"],
+                                a["best"], a["s"], a["ws"], a["wsb"], None)
+    E = w4.W4_ERR_INVALID_ARG
+    assert call(na=1) == E
+    assert call(na=5000) == E
+    assert call(W=0) == E
+    assert call(ws=P + 128) == E                 # workspace not 256-byte aligned
+    assert call(wsb=1024) == E                   # workspace too small
+    assert call(K=500) == E
+    assert call(s=P + 4) == E
