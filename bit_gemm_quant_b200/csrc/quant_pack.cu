@@ -14,10 +14,15 @@
 //   * one resident wave of CTAs; the matrix is a row-major sequence of items
 //     of 32 lane slices of 64 consecutive weights (2048 weights), and warp w
 //     takes items w, w + nwarps, ..., so the warps' shares differ by at most
-//     one item; a warp asks L2 for its item two steps ahead
-//     (cp.async.bulk.prefetch) and reads its slice with four 32-byte loads; a
-//     slice lies in one group (g = 64), in two (g = 32), or in half of one
-//     (g = 128: two lanes);
+//     one item; a slice lies in one group (g = 64), in two (g = 32), or in
+//     half of one (g = 128: two lanes);
+//   * rows of whole slices (K % 64 == 0) are streamed by TMA: each warp keeps
+//     two items in flight in a shared-memory ring (a 32-slice x 128-byte box
+//     with the 128-byte swizzle, so that a lane's eight 16-byte reads of its
+//     slice fall on eight bank groups) and issues the copy of the item after
+//     next as soon as its lanes have read an item; other rows are read with
+//     four 32-byte loads per lane, the item two steps ahead asked into L2
+//     (cp.async.bulk.prefetch);
 //   * group amax / min / max: packed bf16x2 min and max over the lane's raw
 //     words (fp32 comparisons after the fold) and at most one
 //     __shfl_xor_sync; the per-group IEEE divisions (scale and zero point)
@@ -47,6 +52,9 @@
 //   * zero-points of 8 groups are OR-reduced with __shfl_xor_sync across the
 //     4, 8 or 16 lanes that hold them and stored once per word.
 #include "common.cuh"
+#include "tc_ptx.cuh"
+
+#include <cstring>
 
 namespace w4 {
 namespace {
@@ -223,10 +231,45 @@ __device__ __forceinline__ QParams group_params(float a, float mn, float mx, uns
     return q;
 }
 
-template <int G, int MODE, bool FOLD>
+constexpr int kQItemBytes = 32 * 128;              // one item: 32 slices of 64 bf16
+constexpr int kQRingBytes = 8 * 2 * kQItemBytes;   // two items in flight per warp, 8 warps
+constexpr uint64_t kQWaitNs = 200000000ull;        // 200 ms; an item lands in microseconds
+constexpr int kErrQuantWait = 0x401, kErrQuantDrain = 0x402;
+
+// Bounded wait for an item's copy; false after kQWaitNs.
+__device__ __noinline__ bool wait_item(uint32_t bar, uint32_t parity)
+{
+    uint64_t t0 = 0;
+    bool started = false;
+    while (true) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (!started) {
+            t0 = globaltimer();
+            started = true;
+        } else if (globaltimer() - t0 > kQWaitNs) {
+            return false;
+        }
+    }
+}
+
+// With TMA (rows whose length is a multiple of 64), each warp streams its
+// items into a two-item ring in shared memory: a TMA box of 32 slices x 128
+// bytes with the 128-byte swizzle, so that each lane's eight 16-byte reads of
+// its own slice hit eight different bank groups; the copy of the item after
+// next is issued as soon as the lanes have read an item into registers.
+template <int G, int MODE, bool FOLD, bool TMA>
 __global__ void __launch_bounds__(256, 2)
-quant_pack_kernel(const uint32_t *__restrict__ W, int N, int K, const float *__restrict__ s, int s_staged,
-                  uint4 *__restrict__ qweight, unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros)
+quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__restrict__ W, int N, int K,
+                  const float *__restrict__ s, int s_staged, uint4 *__restrict__ qweight,
+                  unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros, int *err)
 {
     constexpr int GPL = (G == 32) ? 2 : 1;       // groups per lane: a lane owns 64 consecutive weights
     constexpr int LPG = (G == 128) ? 2 : 1;      // lanes per group
@@ -236,6 +279,20 @@ quant_pack_kernel(const uint32_t *__restrict__ W, int N, int K, const float *__r
     const int KW = K >> 1;                       // raw words (bf16 pairs) per row
     const int KP = (K + 63) >> 6;                // 64-weight slices per row (the last may hold 32)
     const int NG = K / G, ZW = (NG + 7) >> 3;
+    // dynamic shared memory: [TMA: item rings, 1024-aligned; their barriers] then the staged s
+    extern __shared__ uint8_t qsm[];
+    uint8_t *sbase = TMA ? qsm + ((1024u - (smem_u32(qsm) & 1023u)) & 1023u) : qsm;
+    float4 *s_sm = (float4 *)(sbase + (TMA ? kQRingBytes + 1024 : 0));
+    const int wib = (int)(threadIdx.x >> 5);     // warp in block
+    const uint32_t ring0 = smem_u32(sbase) + wib * 2 * kQItemBytes;
+    const uint32_t bar0 = smem_u32(sbase + kQRingBytes) + wib * 16;
+    if (TMA && lane == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_w) : "memory");
+    }
+    __syncwarp();
     pdl_wait();                                  // the previous kernel's writes are visible
     pdl_launch_dependents();
 
@@ -243,7 +300,6 @@ quant_pack_kernel(const uint32_t *__restrict__ W, int N, int K, const float *__r
     // once per block: slice c (64 factors, 16 float4) is rotated by c % 8
     // float4, so that the 32 lanes' reads of "their" float4 i hit 8 different
     // 16-byte bank groups (the slices are 256 bytes apart).
-    extern __shared__ float4 s_sm[];
     if (FOLD && s_staged) {
         const int n4 = K >> 2, n4p = 16 * ((K + 63) >> 6);   // a half slice at the end is padded with 0
         for (int j = threadIdx.x; j < n4p; j += blockDim.x) {
@@ -273,33 +329,75 @@ quant_pack_kernel(const uint32_t *__restrict__ W, int N, int K, const float *__r
             prefetch_l2(W + (size_t)row * KW + w0, (size_t)min(1024, KW - w0) * 4);
         }
     };
+    // lane 0 (TMA): the item (row, item) into ring slot sl
+    auto issue = [&](int row, int item, int sl) {
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar0 + 8 * sl),
+                     "r"(kQItemBytes)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+            "[%2];" ::"r"(ring0 + sl * kQItemBytes),
+            "l"(&tmap_w), "r"(bar0 + 8 * sl), "r"(0), "r"(row * KP + 32 * item)
+            : "memory");
+    };
     int n = warp0 / IPR, it = warp0 % IPR;       // row and item-in-row of the current item
     int pn = n, pit = it;                        // the item two steps ahead
     advance(pn, pit);
     if (lane == 0) {
-        prefetch_item(n, it);
-        prefetch_item(pn, pit);
+        if (TMA) {
+            if (n < N) issue(n, it, 0);
+            if (pn < N) issue(pn, pit, 1);
+        } else {
+            prefetch_item(n, it);
+            prefetch_item(pn, pit);
+        }
     }
     advance(pn, pit);
 
+    int j = 0;                                   // items of this warp so far
+    bool ok = true;
     while (n < N) {
-        if (lane == 0) prefetch_item(pn, pit);
-        advance(pn, pit);
+        if (!TMA && lane == 0) prefetch_item(pn, pit);
         const int cp = 32 * it + lane;           // this lane's slice
         const bool valid = cp < KP;
         const int cpl = valid ? cp : KP - 1;     // a lane past the row end reads the last slice (not stored)
         const bool valid1 = 64 * cpl + 32 < K;   // the slice's second 32-weight chunk is in the row
         const uint32_t *src = W + (size_t)n * KW + 32 * cpl;
         uint32_t cur[32];
-        ld32<FOLD>((const uint4 *)src, *(uint32_t(*)[8]) & cur[0]);
-        ld32<FOLD>((const uint4 *)(src + 8), *(uint32_t(*)[8]) & cur[8]);
-        if (valid1) {
-            ld32<FOLD>((const uint4 *)(src + 16), *(uint32_t(*)[8]) & cur[16]);
-            ld32<FOLD>((const uint4 *)(src + 24), *(uint32_t(*)[8]) & cur[24]);
-        } else {
+        if (TMA) {
+            // this lane's slice is row `lane` of the box (a lane past the row end
+            // reads the next row's slice, or zeros past the matrix: not stored)
+            const int sl = j & 1;
+            if (!__all_sync(0xffffffffu, wait_item(bar0 + 8 * sl, (uint32_t)(j >> 1) & 1u))) {
+                ok = false;
+                break;
+            }
+            const uint8_t *row = sbase + (ring0 - smem_u32(sbase)) + sl * kQItemBytes + lane * 128;
 #pragma unroll
-            for (int i = 16; i < 32; ++i) cur[i] = 0u;
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = *(const uint4 *)(row + ((c ^ (lane & 7)) << 4));
+                cur[4 * c] = v.x;
+                cur[4 * c + 1] = v.y;
+                cur[4 * c + 2] = v.z;
+                cur[4 * c + 3] = v.w;
+            }
+            __syncwarp();                        // the slot is read: the item after next may land in it
+            if (lane == 0 && pn < N) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                issue(pn, pit, sl);
+            }
+        } else {
+            ld32<FOLD>((const uint4 *)src, *(uint32_t(*)[8]) & cur[0]);
+            ld32<FOLD>((const uint4 *)(src + 8), *(uint32_t(*)[8]) & cur[8]);
+            if (valid1) {
+                ld32<FOLD>((const uint4 *)(src + 16), *(uint32_t(*)[8]) & cur[16]);
+                ld32<FOLD>((const uint4 *)(src + 24), *(uint32_t(*)[8]) & cur[24]);
+            } else {
+#pragma unroll
+                for (int i = 16; i < 32; ++i) cur[i] = 0u;
+            }
         }
+        advance(pn, pit);
         // with a smoothing fold: the 64 weights w' = fl32(w * s), once per item
         float2 xf[FOLD ? 32 : 1];
         if (FOLD) {
@@ -455,44 +553,86 @@ quant_pack_kernel(const uint32_t *__restrict__ W, int N, int K, const float *__r
             if (valid && (lane & (LPW - 1)) == 0) qzeros[(size_t)n * ZW + cp / LPW] = z;
         }
         advance(n, it);
+        ++j;
+    }
+    if (TMA && !ok && lane == 0) {
+        // an item never landed: record it and wait (bounded) for this warp's
+        // copies still in flight (items j and j + 1 at most)
+        atomicCAS(err, 0, kErrQuantWait);
+        int dn = n, dit = it;
+        for (int k = j; k < j + 2 && dn < N; ++k) {
+            if (!wait_item(bar0 + 8 * (k & 1), (uint32_t)(k >> 1) & 1u)) atomicCAS(err, 0, kErrQuantDrain);
+            advance(dn, dit);
+        }
     }
 }
 
 constexpr int kMaxStagedS = 64 * 1024;          // bytes of smoothing factors staged in shared memory
 
-template <int G, int MODE>
-cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, uint32_t *qweight, void *scales,
-                          uint32_t *qzeros, cudaStream_t stream)
+template <int G, int MODE, bool FOLD, bool TMA>
+cudaError_t launch_variant(const CUtensorMap &map, const void *W, int64_t N, int64_t K, const float *s, int staged,
+                           size_t smem, uint32_t *qweight, void *scales, uint32_t *qzeros, int *err,
+                           cudaStream_t stream)
 {
     const int threads = 256;
-    static int per_sm = 0;                       // resident blocks per SM of this instantiation
-    if (per_sm == 0) {
-        const cudaError_t e = s ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_pack_kernel<G, MODE, true>, threads, 0)
-                                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_pack_kernel<G, MODE, false>, threads, 0);
-        if (e != cudaSuccess || per_sm < 1) per_sm = 1;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(quant_pack_kernel<G, MODE, FOLD, TMA>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   2048 + kQRingBytes + kMaxStagedS);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
     }
+    int per_sm = 0;                              // resident blocks per SM at this shared-memory size
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_pack_kernel<G, MODE, FOLD, TMA>, threads, smem) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
     const int64_t items = N * ((K / 64 + 1 + 31) / 32);   // 2048-weight items (upper bound)
     int64_t blocks = (items + 7) / 8;            // one warp per item at most
     const int64_t cap = (int64_t)kNumSMs * per_sm;   // one resident wave; warps stride over rows
     if (blocks > cap) blocks = cap;
+    return launch_pdl(quant_pack_kernel<G, MODE, FOLD, TMA>, dim3((unsigned)blocks), dim3(threads), smem, stream, map,
+                      (const uint32_t *)W, (int)N, (int)K, s, staged, (uint4 *)qweight, (unsigned short *)scales,
+                      qzeros, err);
+}
+
+template <int G, int MODE>
+cudaError_t launch_g_mode(const void *W, int64_t N, int64_t K, const float *s, uint32_t *qweight, void *scales,
+                          uint32_t *qzeros, cudaStream_t stream)
+{
+    int *err = device_error_word();
+    if (!err) return cudaErrorUnknown;
+    // TMA for rows of whole 64-weight slices: W as [N K / 64 slices][64 bf16]
+    CUtensorMap map;
+    memset(&map, 0, sizeof(map));
+    bool tma = (K % 64 == 0) && N * (K / 64) <= (int64_t)INT32_MAX && ((uintptr_t)W % 16) == 0;
+    if (tma) {
+        EncodeTiledFn enc = encode_fn();
+        const cuuint64_t gdim[2] = {64u, (cuuint64_t)(N * (K / 64))};
+        const cuuint64_t gstride[1] = {128u};
+        const cuuint32_t box[2] = {64u, 32u};
+        const cuuint32_t estride[2] = {1u, 1u};
+        tma = enc && enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(W), gdim, gstride, box, estride,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    const size_t ring = tma ? (size_t)1024 + kQRingBytes + 1024 : 0;   // alignment slack, rings, barriers
     if (s) {
         // the smoothing vector in shared memory when it fits in 64 KB
-        static bool attr_set = false;
-        if (!attr_set) {
-            const cudaError_t e = cudaFuncSetAttribute(quant_pack_kernel<G, MODE, true>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxStagedS);
-            if (e != cudaSuccess) return e;
-            attr_set = true;
-        }
         const size_t sbytes = (size_t)((K + 63) / 64) * 256;   // whole 64-factor slices
         const int staged = (sbytes <= (size_t)kMaxStagedS) ? 1 : 0;
-        return launch_pdl(quant_pack_kernel<G, MODE, true>, dim3((unsigned)blocks), dim3(threads),
-                          staged ? sbytes : 0, stream, (const uint32_t *)W, (int)N, (int)K, s, staged,
-                          (uint4 *)qweight, (unsigned short *)scales, qzeros);
+        const size_t smem = ring + (staged ? sbytes : 0);
+        if (tma)
+            return launch_variant<G, MODE, true, true>(map, W, N, K, s, staged, smem, qweight, scales, qzeros, err,
+                                                       stream);
+        return launch_variant<G, MODE, true, false>(map, W, N, K, s, staged, smem, qweight, scales, qzeros, err,
+                                                    stream);
     }
-    return launch_pdl(quant_pack_kernel<G, MODE, false>, dim3((unsigned)blocks), dim3(threads), 0, stream,
-                      (const uint32_t *)W, (int)N, (int)K, (const float *)nullptr, 0, (uint4 *)qweight,
-                      (unsigned short *)scales, qzeros);
+    if (tma)
+        return launch_variant<G, MODE, false, true>(map, W, N, K, nullptr, 0, ring, qweight, scales, qzeros, err,
+                                                    stream);
+    return launch_variant<G, MODE, false, false>(map, W, N, K, nullptr, 0, 0, qweight, scales, qzeros, err, stream);
 }
 
 }  // namespace
