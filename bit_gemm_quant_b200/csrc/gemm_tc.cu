@@ -88,6 +88,53 @@ __device__ __noinline__ bool wait_drain(uint64_t *bar, uint32_t parity)
     return true;
 }
 
+// Bounded wait until both barriers have completed the phase with the given
+// parity; each round tests both at once (their latencies overlap).
+__device__ __noinline__ bool wait_pair_bounded(uint64_t *a, uint64_t *b, uint32_t parity, volatile int *abort_flag)
+{
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        const bool ra = mbar_test(a, parity), rb = mbar_test(b, parity);
+        if (ra && rb) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicCAS(&g_device_error, 0, kErrWaitFullA);
+            return false;
+        }
+    }
+}
+
+// One k-block (four 128 x BN x 16 MMAs, A from tensor memory at a_tmem, B
+// from the SW128 descriptor bdesc, accumulate unless acc0 == 0 for the first)
+// and its commit to `empty`, with non-blocking tests of the next k-block's
+// barriers issued first; returns whether both were complete.
+__device__ __forceinline__ bool mma_kblock_test_next(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                     uint32_t acc0, uint64_t *empty, uint64_t *next_a,
+                                                     uint64_t *next_b, uint32_t next_parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred pa, pb, p0, p1;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 pa, [%1], %3;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 pb, [%2], %3;\n\t"
+        "setp.ne.b32 p0, %8, 0;\n\t"
+        "setp.eq.b32 p1, %8, %8;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%4], [%5], %6, %7, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%4], [%9], %10, %7, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%4], [%11], %12, %7, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%4], [%13], %14, %7, p1;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%15];\n\t"
+        "and.pred pa, pa, pb;\n\t"
+        "selp.u32 %0, 1, 0, pa;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(next_a)), "r"(smem_u32(next_b)), "r"(next_parity), "r"(d_tmem), "r"(a_tmem), "l"(bdesc),
+          "r"(idesc), "r"(acc0), "r"(a_tmem + 8), "l"(bdesc + 2), "r"(a_tmem + 16), "l"(bdesc + 4), "r"(a_tmem + 24),
+          "l"(bdesc + 6), "r"(smem_u32(empty))
+        : "memory");
+    return ok != 0;
+}
+
 template <int BN>
 struct TcCfg {
     static constexpr int kCols = (BN <= 128) ? 256 : 512;               // tensor-memory allocation
@@ -180,19 +227,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ---
         if (lane == 0) {
+            // Per k-block: the four MMAs and the commit are issued in one
+            // block of PTX together with non-blocking tests of the NEXT
+            // k-block's two barriers, whose shared-memory latency (hundreds of
+            // cycles under load) then overlaps the MMA issue instead of
+            // leaving the tensor pipe idle (tcgen05.mma issue blocks until the
+            // previous MMA is nearly done, so the issuer has no slack).
+            bool ok = true, ready = false;
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
-                if (!wait_bounded(&full_a[s], ph, abort_flag, kErrWaitFullA)) break;
-                if (!wait_bounded(&full_b[s], ph, abort_flag, kErrWaitTma)) break;
+                if (!ready) ready = wait_pair_bounded(&full_a[s], &full_b[s], ph, abort_flag);
+                if (!ready) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
+                const int i1 = (i + 1 < nkb) ? i + 1 : i;   // (the last k-block re-tests its own, complete, barriers)
                 const uint64_t bdesc = desc_k_sw128(smem_u32(sB + s * C::kStageBytes));
-#pragma unroll
-                for (int kk = 0; kk < kKB / 16; ++kk)
-                    mma_ts(tmem, tmem + C::kACol0 + s * 32 + kk * 8, bdesc + (uint64_t)(kk * 2), C::kIdesc,
-                           (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&empty[s]);
+                ready = mma_kblock_test_next(tmem, tmem + C::kACol0 + s * 32, bdesc, C::kIdesc, i > 0 ? 1u : 0u,
+                                             &empty[s], &full_a[i1 % kStages], &full_b[i1 % kStages],
+                                             (i1 / kStages) & 1);
             }
+            (void)ok;
             mma_commit(done);
             wait_drain(done, 0);   // no MMA may still be running when tensor memory is freed
         }
