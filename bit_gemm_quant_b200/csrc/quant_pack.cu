@@ -141,9 +141,9 @@ struct QParams {
 // flags marks packed word w (8 weights) if any of its residuals reaches half a
 // step (|rho| >= s16 / 2): exact ties of the quotient and roundings the
 // approximation got wrong.  With CLAMP the asymmetric codes are clamped to
-// [0, 15] before packing (a code of -1 or 16 would borrow from or carry into
-// the neighbouring nibble); without it the caller has shown that every y lies
-// in range.  The arithmetic runs on pairs (fma / add of two fp32 lanes per
+// [0, 15] after the residual is taken and before packing (a code of -1 or 16
+// would borrow from or carry into the neighbouring nibble); without it the
+// caller has shown that every y lies in range.  The arithmetic runs on pairs (fma / add of two fp32 lanes per
 // instruction, each correctly rounded).  With FOLD, xf holds the chunk's 16
 // folded weight pairs (w * s in fp32) and cur is not read.
 template <int MODE, bool FOLD, bool CLAMP>
@@ -162,13 +162,16 @@ __device__ __forceinline__ uint32_t encode(const uint32_t *cur, const float2 *xf
             const int p = 4 * w + j;
             const float2 x = FOLD ? xf[p] : weight_pair<false>(cur[p], make_float2(1.f, 1.f));
             float2 y = __ffma2_rn(x, inv2, mg2);
+            // the residual of the unclamped rounding: clip(rint(w'/s16) + zp)
+            // only needs rint itself to be exact, so a weight that the clamp
+            // moves (the group maximum may round to 16) is not flagged
+            const float2 r = __fadd2_rn(y, nmg2);
+            const float2 rho = __ffma2_rn(r, nd2, x);
+            m = fmaxf(m, fmaxf(fabsf(rho.x), fabsf(rho.y)));
             if (MODE == W4_ASYM && CLAMP) {
                 y.x = fmaxf(fminf(y.x, q.ymax), kMagic);
                 y.y = fmaxf(fminf(y.y, q.ymax), kMagic);
             }
-            const float2 r = __fadd2_rn(y, nmg2);
-            const float2 rho = __ffma2_rn(r, nd2, x);
-            m = fmaxf(m, fmaxf(fabsf(rho.x), fabsf(rho.y)));
             yb[2 * j] = __float_as_uint(y.x);
             yb[2 * j + 1] = __float_as_uint(y.y);
         }
