@@ -168,7 +168,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     using C = TcCfg<BN>;
     constexpr int kStages = C::kStages;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // (an offset from the shared array, not an integer cast, so that the
+    // compiler keeps the shared address space and emits shared loads/stores)
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *sB = smem;                                               // kStages x BN x 128 bytes
     uint64_t *full_b = (uint64_t *)(smem + kStages * C::kStageBytes);
     uint64_t *full_a = full_b + kStages;
@@ -233,23 +235,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             // cycles under load) then overlaps the MMA issue instead of
             // leaving the tensor pipe idle (tcgen05.mma issue blocks until the
             // previous MMA is nearly done, so the issuer has no slack).
-            bool ok = true, ready = false;
+            bool ready = false;
+            int s = 0;
+            uint32_t ph = 0;
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
                 if (!ready) ready = wait_pair_bounded(&full_a[s], &full_b[s], ph, abort_flag);
-                if (!ready) {
-                    ok = false;
-                    break;
-                }
+                if (!ready) break;
                 tc_fence_after();
-                const int i1 = (i + 1 < nkb) ? i + 1 : i;   // (the last k-block re-tests its own, complete, barriers)
+                // the next k-block's stage and phase (the last k-block re-tests its own, complete, barriers)
+                int s1 = s + 1;
+                uint32_t ph1 = ph;
+                if (s1 == kStages) {
+                    s1 = 0;
+                    ph1 ^= 1u;
+                }
+                if (i + 1 == nkb) {
+                    s1 = s;
+                    ph1 = ph;
+                }
                 const uint64_t bdesc = desc_k_sw128(smem_u32(sB + s * C::kStageBytes));
                 ready = mma_kblock_test_next(tmem, tmem + C::kACol0 + s * 32, bdesc, C::kIdesc, i > 0 ? 1u : 0u,
-                                             &empty[s], &full_a[i1 % kStages], &full_b[i1 % kStages],
-                                             (i1 / kStages) & 1);
+                                             &empty[s], &full_a[s1], &full_b[s1], ph1);
+                s = s1;
+                ph = ph1;
             }
-            (void)ok;
             mma_commit(done);
             wait_drain(done, 0);   // no MMA may still be running when tensor memory is freed
         }
@@ -275,13 +284,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             const int kq = (kb_begin + i) * 2;       // first 32-weight half of this k-block
             const bool ok0 = okn && kq < KQ, ok1 = okn && (kq + 1 < KQ);
             const int j0 = (kq * 32) >> group_log2, j1 = ((kq + 1) * 32) >> group_log2;
+            // (with g >= 64 both halves of a k-block lie in one group: j1 == j0)
             sd.s0 = ok0 ? __ldg(srow + j0) : (unsigned short)0;
-            sd.s1 = ok1 ? __ldg(srow + j1) : (unsigned short)0;
-            if (asym) {
-                sd.z0 = ok0 ? (__ldg(zrow + (j0 >> 3)) >> (4 * (j0 & 7))) & 0xFu : 0u;
-                sd.z1 = ok1 ? (__ldg(zrow + (j1 >> 3)) >> (4 * (j1 & 7))) & 0xFu : 0u;
+            sd.z0 = !asym ? 8u : ok0 ? (__ldg(zrow + (j0 >> 3)) >> (4 * (j0 & 7))) & 0xFu : 0u;
+            if (group_log2 == 5) {
+                sd.s1 = ok1 ? __ldg(srow + j1) : (unsigned short)0;
+                sd.z1 = !asym ? 8u : ok1 ? (__ldg(zrow + (j1 >> 3)) >> (4 * (j1 & 7))) & 0xFu : 0u;
             } else {
-                sd.z0 = sd.z1 = 8u;
+                sd.s1 = ok1 ? sd.s0 : (unsigned short)0;
+                sd.z1 = ok1 ? sd.z0 : 0u;
             }
         };
 #pragma unroll
@@ -289,13 +300,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             if (h + 2 * d < nkb) fetch(h + 2 * d, buf[d]);
 
         bool ok = true;
+        int s = h;                                   // stage and phase of k-block i (i = h, h + 2, ...; kStages is even)
+        uint32_t ph = 0;
+        static_assert(kStages % 2 == 0, "the dequantizing warps step two stages at a time");
         for (int i0 = h; i0 < nkb && ok; i0 += 2 * D) {
 #pragma unroll
             for (int d = 0; d < D; ++d) {
                 const int i = i0 + 2 * d;
                 if (i >= nkb || !ok) break;
-                const int s = i % kStages;
-                const uint32_t ph = (i / kStages) & 1;
                 // full_b also means the MMAs of this stage's previous round are done
                 // (the producer refilled it only after their commit), so its
                 // tensor-memory A columns are free
@@ -308,7 +320,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 const uint4 w0 = cs[0], w1 = cs[1];
                 uint32_t v[32];
                 const GroupConst c0 = group_const(buf[d].s0, buf[d].z0);
-                const GroupConst c1 = group_const(buf[d].s1, buf[d].z1);
+                GroupConst c1 = c0;
+                if (group_log2 == 5 || buf[d].s1 != buf[d].s0 || buf[d].z1 != buf[d].z0)
+                    c1 = group_const(buf[d].s1, buf[d].z1);
                 if (i + 2 * D < nkb) fetch(i + 2 * D, buf[d]);
                 const uint32_t wa[4] = {w0.x, w0.y, w0.z, w0.w};
                 const uint32_t wb[4] = {w1.x, w1.y, w1.z, w1.w};
@@ -324,6 +338,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full_a[s]);
+                s += 2;
+                if (s >= kStages) {
+                    s -= kStages;
+                    ph ^= 1u;
+                }
             }
         }
 
