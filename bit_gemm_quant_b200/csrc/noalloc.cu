@@ -2,11 +2,10 @@
 // device memory.
 //
 // Who needs it: code that runs where cudaMalloc is not available or not
-// allowed -- inside a CUDA-graph capture that must not allocate, under a
-// framework whose caching allocator owns all device memory and forbids
-// side allocations, in a real-time or embedded host that freezes its memory
-// map after start-up, or in a plug-in that receives only its input and output
-// buffers.  w4a16_gemm needs a caller-provided workspace for its split-K
+// allowed -- under a framework whose caching allocator owns all device memory
+// and forbids side allocations, in a real-time or embedded host that freezes
+// its memory map after start-up, or in a plug-in that receives only its input
+// and output buffers.  w4a16_gemm needs a caller-provided workspace for its split-K
 // shapes; this entry point uses a fixed scratch array that the library itself
 // owns instead, so the caller passes only inputs and outputs.
 //

@@ -43,7 +43,8 @@
  * Conventions for every entry point:
  *   - All data pointers are DEVICE pointers owned by the caller, 16-byte
  *     aligned unless stated otherwise; the library allocates no device memory
- *     and keeps no state between calls.
+ *     and keeps no state between calls (except w4a16_gemm_noalloc's fixed
+ *     scratch array, described there).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
  *     stream).  Calls are asynchronous: the library never synchronizes.
  *   - Arguments are validated on the host before anything is launched; a
@@ -162,9 +163,9 @@ w4_status w4_awq_search(const void *W, const void *X, int64_t N, int64_t K, int6
 
 /*
  * w4a16_gemm_noalloc -- w4a16_gemm for callers that cannot allocate device
- * memory (a stream capture that must not allocate, a host whose allocator
- * owns all device memory, a plug-in that only receives its input and output
- * buffers).  The pages have no counterpart to this entry point: it only
+ * memory (a host whose allocator owns all device memory, a real-time host
+ * that freezes its memory map after start-up, a plug-in that only receives its
+ * input and output buffers).  The pages have no counterpart to this entry point: it only
  * changes where the split-K scratch lives.
  *   Arguments, results and errors are those of w4a16_gemm without the
  *   workspace.  The split-K scratch is a library-owned device array of
