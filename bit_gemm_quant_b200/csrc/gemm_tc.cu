@@ -28,6 +28,13 @@
 // k-block) and then run the epilogue.  A 4- or 6-stage ring couples them with
 // mbarriers: full_b (TMA bytes landed), full_a (4 warps stored their A
 // slice), empty (tcgen05.commit: the MMAs that read the stage are done).
+// tcgen05.mma issue blocks until the previous MMA is nearly done, so the
+// issuer never checks a barrier between two k-blocks on its own: the
+// non-blocking tests of the next k-block's barriers go in the same block of
+// PTX as the current k-block's MMAs, and their latency overlaps the MMAs.
+// For the same reason the dequantizing loop is kept lean: two dequantizing
+// warps share the issuer's sub-partition (tensor-memory lane quarters follow
+// the warp index), and every instruction they issue can delay the next MMA.
 // Every wait is bounded in time; a wait that runs out records an error code
 // (read by w4_device_error), raises a CTA-wide abort flag, and the CTA drains
 // its own in-flight copies and MMAs, frees its tensor memory and returns.
