@@ -110,6 +110,19 @@ def problems_for(workload: str):
     return [(p.name, p) for p in probs]
 
 
+WORKLOAD_DESC = {
+    "decode": "decode GEMV: M=1, K=4096, N in {4096,11008,12288}, asymmetric INT4 g=128, fp16 scales, uint4 zero-points; step = w4_quant_pack + w4a16_gemm per layer",
+    "smallbatch": "small-batch decode: K=8192, N=28672, symmetric INT4 g=128, M in {2,4,8,16,32}; step = 1 w4_quant_pack + 5 w4a16_gemm",
+    "prefill": "prefill GEMM: K=4096, N=14336, asymmetric INT4 g=128, M in {512,2048,8192}; step = 1 w4_quant_pack + 3 w4a16_gemm",
+    "quantizer": "quantizer sweep: W[28672,8192], g in {32,64,128} x {sym,asym} + smoothing fold; step = 7 w4_quant_pack",
+}
+
+
+def awq_desc(M, N, K, g, na):
+    return ("AWQ scale search: W[%d,%d] bf16, X[%d,%d] calibration rows with 1%% outlier channels x20, "
+            "asymmetric INT4 g=%d, %d alphas; step = one whole search" % (N, K, M, K, g, na))
+
+
 def kernel_name(M: int) -> str:
     return "w4a16_gemv" if M <= 16 else "w4a16_gemm_tc"
 
@@ -467,12 +480,7 @@ def run_w4(args, rank, world, local_rank):
         cpu = cpu_baseline(args.workload, plist, keys, qp, host_W, host_X, host_s, args.cpu_budget)
 
     if rank == 0:
-        wl_desc = {
-            "decode": "decode GEMV: M=1, K=4096, N in {4096,11008,12288}, asymmetric INT4 g=128, fp16 scales, uint4 zero-points; step = w4_quant_pack + w4a16_gemm per layer",
-            "smallbatch": "small-batch decode: K=8192, N=28672, symmetric INT4 g=128, M in {2,4,8,16,32}; step = 1 w4_quant_pack + 5 w4a16_gemm",
-            "prefill": "prefill GEMM: K=4096, N=14336, asymmetric INT4 g=128, M in {512,2048,8192}; step = 1 w4_quant_pack + 3 w4a16_gemm",
-            "quantizer": "quantizer sweep: W[28672,8192], g in {32,64,128} x {sym,asym} + smoothing fold; step = 7 w4_quant_pack",
-        }[args.workload]
+        wl_desc = WORKLOAD_DESC[args.workload]
         out = {
             "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": K,
             "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / K, 5),
@@ -597,6 +605,8 @@ def run_reference(args, rank, world):
         return
     import oracle
     oracle.build()
+    if args.workload == "awq":
+        return run_reference_awq(args, world)
     plist = problems_for(args.workload)
     keys = list(dict.fromkeys(k for k, _ in plist))
     first = {k: p for k, p in reversed(plist)}
@@ -619,13 +629,40 @@ def run_reference(args, rank, world):
         val, unit = nb / dt / 1e9, "GB/s"
     sample = ("%d rows of each weight per step (rotating): oracle fold+quantize+pack, dequantize and fp64 "
               "product for those output channels, single thread" % rows)
+    print_reference(args, world, val, unit, dt * 1e3 / args.steps, WORKLOAD_DESC[args.workload], sample)
+
+
+def print_reference(args, world, val, unit, ms_per_step, desc, sample):
     out = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
-           "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": dt * 1e3 / args.steps,
+           "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
-           "data": "synthetic", "config": {"workload": args.workload, "kind": "CPU oracle on a bounded sample"},
+           "data": "synthetic", "config": {"workload": desc, "kind": "CPU oracle on a bounded sample"},
            "cpu_baseline": {"value": val, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
+
+
+def run_reference_awq(args, world):
+    """The oracle's AWQ search over the first `rows` output channels of the
+    bench's layer (all 20 alphas, all calibration rows), single thread; the
+    algorithmic bytes are those of a search over that many channels."""
+    import oracle.awq as oawq
+    sh = AWQ_SHAPE
+    M, N, K, g, mode, na = sh["M"], sh["N"], sh["K"], sh["group"], sh["mode"], sh["n_alpha"]
+    rows = 8
+    W = synth.weights(21, N, K, 0.02, 0.01, 5.0)
+    X = synth.activations(22, M, K, 0.01, 20.0)
+    for si in range(max(3, args.warmup)):
+        oawq.awq_losses(W[(si * rows) % N:(si * rows) % N + rows], X, g, mode, na)
+    t0 = time.perf_counter()
+    for si in range(args.steps):
+        r0 = (si * rows) % N
+        oawq.awq_losses(W[r0:r0 + rows], X, g, mode, na)
+    dt = time.perf_counter() - t0
+    val = args.steps * awq_bytes(M, rows, K, g, mode, na) / dt / 1e9
+    sample = ("the search over %d output channels per step (rotating), all %d calibration rows and %d alphas: "
+              "oracle fold+quantize+pack, dequantize, fp64 products and losses, single thread" % (rows, M, na))
+    print_reference(args, world, val, "GB/s", dt * 1e3 / args.steps, awq_desc(M, N, K, g, na), sample)
 
 
 # ------------------------------------------------------------ awq search --
@@ -712,9 +749,7 @@ def run_awq(args, rank, world, local_rank):
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K_steps,
             "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / K_steps, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "AWQ scale search: W[%d,%d] bf16, X[%d,%d] calibration rows with 1%% outlier "
-                                   "channels x20, asymmetric INT4 g=%d, %d alphas; step = one whole search"
-                                   % (N, K, M, K, g, na),
+            "config": {"workload": awq_desc(M, N, K, g, na),
                        "timing": "K searches captured in one CUDA graph, replayed between CUDA events after 1.5 s "
                                  "of untimed replays; max over ranks",
                        "parallelism": "replicas (dp%d), no data-path collective" % world},
