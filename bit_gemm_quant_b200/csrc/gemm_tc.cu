@@ -223,7 +223,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
-                if (!wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyTma)) break;
+                if (!mbar_try_wait(&empty[s], ph ^ 1) && !wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyTma))
+                    break;
                 mbar_arrive_expect_tx(&full_b[s], C::kStageBytes);
                 tma_load_2d(sB + s * C::kStageBytes, &tmap_x, &full_b[s], (kb_begin + i) * kKB, m0);
                 tma_load_2d(sB + s * C::kStageBytes + C::kBBytes, &tmap_q, &full_b[s], (kb_begin + i) * 8, n0);
@@ -318,7 +319,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 // full_b also means the MMAs of this stage's previous round are done
                 // (the producer refilled it only after their commit), so its
                 // tensor-memory A columns are free
-                if (!__all_sync(0xffffffffu, wait_bounded(&full_b[s], ph, abort_flag, kErrWaitEmptyDeq))) {
+                // (the inline try_wait is the usual case: the stage landed long ago)
+                if (!__all_sync(0xffffffffu, mbar_try_wait(&full_b[s], ph) ||
+                                                 wait_bounded(&full_b[s], ph, abort_flag, kErrWaitEmptyDeq))) {
                     ok = false;
                     break;
                 }
