@@ -243,29 +243,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             // cycles under load) then overlaps the MMA issue instead of
             // leaving the tensor pipe idle (tcgen05.mma issue blocks until the
             // previous MMA is nearly done, so the issuer has no slack).
-            bool ready = false;
-            int s = 0;
+            // The loop is unrolled over the ring's stages, so that the stage,
+            // its descriptor offset and its barriers are constants: between two
+            // k-blocks the issuer runs only a handful of instructions.
+            bool ready = false, stop = false;
             uint32_t ph = 0;
-            for (int i = 0; i < nkb; ++i) {
-                if (!ready) ready = wait_pair_bounded(&full_a[s], &full_b[s], ph, abort_flag);
-                if (!ready) break;
-                tc_fence_after();
-                // the next k-block's stage and phase (the last k-block re-tests its own, complete, barriers)
-                int s1 = s + 1;
-                uint32_t ph1 = ph;
-                if (s1 == kStages) {
-                    s1 = 0;
-                    ph1 ^= 1u;
+            const uint64_t bdesc0 = desc_k_sw128(smem_u32(sB));
+            const uint32_t a0 = tmem + C::kACol0;
+            for (int i0 = 0; i0 < nkb && !stop; i0 += kStages, ph ^= 1u) {
+#pragma unroll
+                for (int st = 0; st < kStages; ++st) {
+                    const int i = i0 + st;
+                    if (i >= nkb) break;
+                    if (!ready) ready = wait_pair_bounded(&full_a[st], &full_b[st], ph, abort_flag);
+                    if (!ready) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    // the next k-block's stage and phase (the last k-block re-tests its own, complete, barriers)
+                    const int s1 = (st + 1 == kStages) ? 0 : st + 1;
+                    const uint32_t ph1 = (st + 1 == kStages) ? (ph ^ 1u) : ph;
+                    const bool last = i + 1 == nkb;
+                    ready = mma_kblock_test_next(tmem, a0 + st * 32,
+                                                 bdesc0 + (uint64_t)((st * C::kStageBytes) >> 4), C::kIdesc,
+                                                 i > 0 ? 1u : 0u, &empty[st], last ? &full_a[st] : &full_a[s1],
+                                                 last ? &full_b[st] : &full_b[s1], last ? ph : ph1);
                 }
-                if (i + 1 == nkb) {
-                    s1 = s;
-                    ph1 = ph;
-                }
-                const uint64_t bdesc = desc_k_sw128(smem_u32(sB + s * C::kStageBytes));
-                ready = mma_kblock_test_next(tmem, tmem + C::kACol0 + s * 32, bdesc, C::kIdesc, i > 0 ? 1u : 0u,
-                                             &empty[s], &full_a[s1], &full_b[s1], ph1);
-                s = s1;
-                ph = ph1;
             }
             mma_commit(done);
             wait_drain(done, 0);   // no MMA may still be running when tensor memory is freed
