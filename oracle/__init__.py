@@ -24,6 +24,8 @@ _SO = os.path.join(_HERE, "libw4oracle.so")
 _lib = None
 
 SYM, ASYM = 0, 1
+NVFP4, MXFP4 = 0, 1          # block-scaled FP4 kinds: 16-weight blocks with E4M3 scales, 32 with E8M0
+FP4_BLOCK = {NVFP4: 16, MXFP4: 32}
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +60,14 @@ def lib() -> ctypes.CDLL:
         L.orc_gemm_f64.argtypes = [P, I64, I64, P, I64, P]
         L.orc_gemm_f64.restype = None
         L.orc_e2m1_decode.argtypes, L.orc_e2m1_decode.restype = [I], ctypes.c_float
+        L.orc_f32_to_e2m1_sat.argtypes, L.orc_f32_to_e2m1_sat.restype = [ctypes.c_float], I
+        L.orc_e4m3_decode.argtypes, L.orc_e4m3_decode.restype = [I], ctypes.c_float
+        L.orc_f32_to_e4m3_sat.argtypes, L.orc_f32_to_e4m3_sat.restype = [ctypes.c_float], I
+        L.orc_e8m0_decode.argtypes, L.orc_e8m0_decode.restype = [I], ctypes.c_float
+        L.orc_fp4_quant_rows.argtypes = [P, I64, I64, I, P, P]
+        L.orc_fp4_quant_rows.restype = I
+        L.orc_fp4_dequant_rows.argtypes = [P, P, I64, I64, I, P]
+        L.orc_fp4_dequant_rows.restype = I
         _lib = L
     return _lib
 
@@ -216,3 +226,57 @@ def w4a16_abs_reference(X_bits, qweight, scales, qzeros, K, g, mode, threads=1):
 def e2m1_decode(code: int) -> float:
     """Value of a 4-bit E2M1 code (page 5 section 2.1)."""
     return float(lib().orc_e2m1_decode(int(code)))
+
+
+# --- block-scaled FP4 (NVFP4 / MXFP4) ----------------------------------------
+# Page 2 (learn.longtimenohack.com .../quantization.html, the Blackwell FP4
+# paragraph): E2M1 values with one FP8 E4M3 scale per 16 weights, amax mapped
+# to 6; page 3 (blog.freezetheflame.cc .../quantization-deep-dive.html, section
+# 4.3): MXFP4, one E8M0 scale per 32 weights; page 5 (ai-infra.cypggs.com
+# .../02-core-ideas, section 2.1): the E2M1 value set and the E4M3 format.  The
+# readings are stated in w4_oracle.c.
+
+def f32_to_e2m1(x: float) -> int:
+    """E2M1 code of x: nearest value, ties to the even fraction bit, |x| > 6 saturating."""
+    return int(lib().orc_f32_to_e2m1_sat(float(x)))
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an FP8 E4M3 code (1+4+3, bias 7, max 448, S.1111.111 NaN)."""
+    return float(lib().orc_e4m3_decode(int(code)))
+
+
+def f32_to_e4m3(x: float) -> int:
+    """E4M3 code of x, round to nearest even, finite overflow saturating to 448."""
+    return int(lib().orc_f32_to_e4m3_sat(float(x)))
+
+
+def e8m0_decode(code: int) -> float:
+    """Value of an E8M0 scale: 2^(code - 127)."""
+    return float(lib().orc_e8m0_decode(int(code)))
+
+
+def fp4_quant(W_bits: np.ndarray, kind: int):
+    """Block-scaled FP4 quantization of bf16 W [N, K] (bit patterns).
+
+    Returns (codes uint8 [N, K/2], two per byte with element 2i in the low
+    nibble; scales uint8 [N, K/block]: E4M3 codes for NVFP4, E8M0 for MXFP4)."""
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    N, K = W_bits.shape
+    B = FP4_BLOCK[kind]
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros((N, K // B), dtype=np.uint8)
+    if lib().orc_fp4_quant_rows(_ptr(W_bits), N, K, kind, _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("K must be a multiple of the block")
+    return codes, scales
+
+
+def fp4_dequant(codes: np.ndarray, scales: np.ndarray, kind: int) -> np.ndarray:
+    """w^ = e2m1(code) * scale as fp32 [N, K] (exact)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    N, K = codes.shape[0], codes.shape[1] * 2
+    out = np.zeros((N, K), dtype=np.float32)
+    if lib().orc_fp4_dequant_rows(_ptr(codes), _ptr(scales), N, K, kind, _ptr(out)) != 0:
+        raise ValueError("K must be a multiple of the block")
+    return out

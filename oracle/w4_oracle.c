@@ -315,3 +315,156 @@ float orc_e2m1_decode(int code)
     double v = (e == 0) ? ldexp((double)f, -1) : ldexp(1.0 + 0.5 * f, e - 1);
     return (float)(s ? -v : v);
 }
+
+/* ------------------------------------------------------------------------ */
+/* FP4 block-scaled weights (NVFP4 and MXFP4).                               */
+/*                                                                           */
+/* Page 2 (learn.longtimenohack.com .../quantization.html, the Blackwell FP4  */
+/* paragraph and its teaching snippet): E2M1 values, blocks of 16 weights     */
+/* sharing one FP8 E4M3 scale, amax mapped to the E2M1 maximum 6, 4 + 8/16 =  */
+/* 4.5 bits per weight.  Page 3 (blog.freezetheflame.cc .../quantization-     */
+/* deep-dive.html, section 4.3): MXFP4, blocks of 32 sharing an E8M0 scale,   */
+/* two FP4 values per byte.  Page 5 (ai-infra.cypggs.com .../02-core-ideas,   */
+/* section 2.1): the E2M1 value set and the E4M3 format (1+4+3, max 448,      */
+/* S.1111.111 is NaN).                                                        */
+/*                                                                           */
+/* Readings where the pages leave a step open:                               */
+/*   NVFP4: s = e4m3_rn(fl32(amax / 6)), codes e2m1_rn(fl32(w / s)); the      */
+/*     snippet's second factor 6.0 is garbled (it would map amax to 36) and   */
+/*     is left out; a block whose s is 0 gets all-zero codes.                 */
+/*   MXFP4: the pages give no exponent rule; the shared scale is            */
+/*     2^(floor(log2 amax) - 2), the OCP Microscaling rule with the E2M1     */
+/*     maximum exponent 2, clamped to the E8M0 range [-127, 127]; an all-    */
+/*     zero block gets 2^-127 and zero codes.                                 */
+/*   Both: elements round to nearest E2M1 value, ties to the even fraction    */
+/*     bit, magnitudes above 6 saturate to 6; scales saturate too (E4M3 at    */
+/*     448).  Codes pack two per byte, element 2i in the low nibble.          */
+/*   Dequantized weight w^ = e2m1(code) * scale, exact in fp32 (at most 6     */
+/*   significant bits), so also exact in bf16 within bf16's range.           */
+/* ------------------------------------------------------------------------ */
+
+/* E4M3 (OCP FP8 "FN"): 1 sign bit, 4 exponent bits with bias 7, 3 fraction
+ * bits; exponent field 0 encodes subnormals f * 2^-9; no infinity; the
+ * all-ones magnitude S.1111.111 is NaN, so the largest finite value is 448. */
+float orc_e4m3_decode(int code)
+{
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, f = code & 7;
+    double v;
+    if (e == 15 && f == 7) v = NAN;
+    else if (e == 0) v = ldexp((double)f, -9);
+    else v = ldexp((double)(8 + f), e - 10);
+    return (float)(s ? -v : v);
+}
+
+/* float -> E4M3 code, round to nearest even; finite magnitudes that round
+ * above 448 (and infinities) saturate to 448, NaN stays NaN. */
+int orc_f32_to_e4m3_sat(float f)
+{
+    uint32_t x = f32_bits(f);
+    int sign = (x >> 31) ? 0x80 : 0;
+    uint32_t ex = (x >> 23) & 0xFFu, fr = x & 0x7FFFFFu;
+    if (ex == 0xFFu) return fr ? (sign | 0x7F) : (sign | 0x7E);
+    if (ex == 0 && fr == 0) return sign;
+    uint64_t m = ex ? (fr | 0x800000u) : fr;
+    int E = ex ? (int)ex - 150 : -149;
+    int qe;
+    uint64_t r = round_sig(m, E, 4, -9, &qe);
+    if (r == 0) return sign;
+    if (r < 8u) return sign | (int)r;                       /* subnormal, qe = -9     */
+    if (r == 16u) { r = 8u; qe += 1; }                      /* carry into exponent    */
+    int bexp = qe + 10;                                     /* r * 2^qe, r in [8, 16) */
+    if (bexp > 15 || (bexp == 15 && r - 8u == 7u)) return sign | 0x7E;
+    return sign | (bexp << 3) | (int)(r - 8u);
+}
+
+/* float -> E2M1 code, round to nearest even (ties to the even fraction bit);
+ * magnitudes above 6 saturate to 6.  Exponent field 0 holds 0 and 0.5. */
+int orc_f32_to_e2m1_sat(float f)
+{
+    uint32_t x = f32_bits(f);
+    int sign = (x >> 31) ? 8 : 0;
+    uint32_t ex = (x >> 23) & 0xFFu, fr = x & 0x7FFFFFu;
+    if (ex == 0xFFu) return sign | 7;
+    if (ex == 0 && fr == 0) return sign;
+    uint64_t m = ex ? (fr | 0x800000u) : fr;
+    int E = ex ? (int)ex - 150 : -149;
+    int qe;
+    uint64_t r = round_sig(m, E, 2, -1, &qe);
+    if (r == 0) return sign;
+    if (r < 2u) return sign | (int)r;                       /* 0.5, qe = -1           */
+    if (r == 4u) { r = 2u; qe += 1; }
+    int e = qe + 2;                                         /* r * 2^qe, r in {2, 3}  */
+    if (e > 3) return sign | 7;
+    return sign | (e << 1) | (int)(r - 2u);
+}
+
+/* E8M0: the power of two 2^(code - 127), code in [0, 254] (255 is NaN). */
+float orc_e8m0_decode(int code)
+{
+    if ((code & 0xFF) == 0xFF) return NAN;
+    return (float)ldexp(1.0, (code & 0xFF) - 127);
+}
+
+/* Block-scaled FP4 quantization of W (bf16 [N, K], K a multiple of the block).
+ * kind 0 = NVFP4 (block 16, E4M3 scales), 1 = MXFP4 (block 32, E8M0 scales).
+ * codes: uint8 [N, K/2], scales: uint8 [N, K/block]. */
+int orc_fp4_quant_rows(const uint16_t *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales)
+{
+    const int64_t B = kind == 0 ? 16 : 32;
+    if (K % B != 0 || (kind != 0 && kind != 1)) return -1;
+    memset(codes, 0, (size_t)(N * (K / 2)));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t b = 0; b < K / B; ++b) {
+            const uint16_t *w = W + n * K + b * B;
+            float amax = 0.0f;
+            for (int64_t i = 0; i < B; ++i) {
+                float a = fabsf(orc_bf16_to_f32(w[i]));
+                if (a > amax) amax = a;
+            }
+            float sc;
+            int scode;
+            if (kind == 0) {
+                volatile float t = amax / 6.0f;                 /* one IEEE division */
+                scode = orc_f32_to_e4m3_sat(t);
+                sc = orc_e4m3_decode(scode);
+            } else {
+                int e = -127;
+                if (amax > 0.0f) {
+                    int ex;
+                    frexp((double)amax, &ex);               /* amax = f 2^ex, f in [0.5, 1) */
+                    e = (ex - 1) - 2;                       /* floor(log2 amax) - 2          */
+                    if (e < -127) e = -127;
+                    if (e > 127) e = 127;
+                }
+                scode = e + 127;
+                sc = orc_e8m0_decode(scode);
+            }
+            scales[n * (K / B) + b] = (uint8_t)scode;
+            for (int64_t i = 0; i < B; ++i) {
+                int q = 0;
+                if (sc > 0.0f) {
+                    volatile float t = orc_bf16_to_f32(w[i]) / sc;   /* one IEEE division */
+                    q = orc_f32_to_e2m1_sat(t);
+                }
+                const int64_t k = b * B + i;
+                codes[n * (K / 2) + k / 2] |= (uint8_t)(q << (4 * (k & 1)));
+            }
+        }
+    }
+    return 0;
+}
+
+/* w^[n][k] = e2m1(code) * scale, fp32 [N, K]. */
+int orc_fp4_dequant_rows(const uint8_t *codes, const uint8_t *scales, int64_t N, int64_t K, int kind, float *out)
+{
+    const int64_t B = kind == 0 ? 16 : 32;
+    if (K % B != 0 || (kind != 0 && kind != 1)) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            const int q = (codes[n * (K / 2) + k / 2] >> (4 * (k & 1))) & 15;
+            const int sc = scales[n * (K / B) + k / B];
+            const double s = kind == 0 ? (double)orc_e4m3_decode(sc) : (double)orc_e8m0_decode(sc);
+            out[n * K + k] = (float)((double)orc_e2m1_decode(q) * s);
+        }
+    return 0;
+}

@@ -1,0 +1,210 @@
+"""Pins of the oracle's block-scaled FP4 quantizers (NVFP4, MXFP4) and of the
+formats they use (E2M1, FP8 E4M3, E8M0).
+
+Each expected value is printed on a page (tests/golden/fp4_formats.json, cited
+there), comes from an independent library routine (torch's float8_e4m3fn), or
+from brute force in exact arithmetic over the formats' value sets.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import golden
+
+NVFP4, MXFP4 = 0, 1
+
+E2M1_VALUES = {0: 0.0, 1: 0.5, 2: 1.0, 3: 1.5, 4: 2.0, 5: 3.0, 6: 4.0, 7: 6.0}   # code & 7 -> magnitude
+
+
+def e2m1_nearest(x: float) -> float:
+    """Nearest E2M1 value to x in exact arithmetic, ties to the even fraction
+    bit (the low bit of the code), by brute force over the eight magnitudes."""
+    fx = Fraction(abs(x))
+    best = None
+    for code, v in E2M1_VALUES.items():
+        d = abs(fx - Fraction(v))
+        key = (d, code & 1)
+        if best is None or key < best[0]:
+            best = (key, v)
+    v = best[1]
+    return -v if x < 0 else v
+
+
+def bf16(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of fp32 values (torch's round to nearest even)."""
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_value(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------------------------ E2M1 --
+
+def test_e2m1_encode_is_nearest_value_ties_to_even(oracle_mod):
+    xs = [i / 64 for i in range(-640, 641)] + [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, 7.0, 100.0, 1e-30]
+    xs += list(np.random.default_rng(3).standard_normal(2000) * 3)
+    for x in xs:
+        x = float(np.float32(x))
+        got = oracle_mod.e2m1_decode(oracle_mod.f32_to_e2m1(x))
+        assert got == e2m1_nearest(x), (x, got, e2m1_nearest(x))
+
+
+def test_e2m1_encode_inverts_decode(oracle_mod):
+    for c in range(16):
+        assert oracle_mod.f32_to_e2m1(oracle_mod.e2m1_decode(c)) == c
+
+
+# ------------------------------------------------------------------ E4M3 --
+
+def test_e4m3_format_facts(oracle_mod):
+    fx = golden("fp4_formats.json")["e4m3"]
+    vals = [oracle_mod.e4m3_decode(c) for c in range(256)]
+    finite = [v for v in vals if v == v]
+    assert max(finite) == fx["max"] and min(finite) == -fx["max"]
+    assert oracle_mod.e4m3_decode(1 << fx["fraction_bits"]) == fx["min_normal"]
+    assert [c for c in range(256) if vals[c] != vals[c]] == fx["nan_codes"]
+
+
+def test_e4m3_decode_matches_torch(oracle_mod):
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    for c in range(256):
+        got = oracle_mod.e4m3_decode(c)
+        assert (got == ref[c]) or (got != got and ref[c] != ref[c]), (c, got, ref[c])
+
+
+def test_e4m3_encode_matches_torch_in_range(oracle_mod):
+    finite = sorted({oracle_mod.e4m3_decode(c) for c in range(128) if c != 127})
+    mids = [(a + b) / 2 for a, b in zip(finite, finite[1:])]
+    rng = np.random.default_rng(7)
+    xs = np.array(finite + mids + list(rng.uniform(-448, 448, 4000)) +
+                  list(rng.standard_normal(4000) * 2.0 ** rng.integers(-12, 8, 4000)), dtype=np.float32)
+    xs = np.concatenate([xs, -xs])
+    xs = xs[np.abs(xs) <= 448]
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle_mod.f32_to_e4m3(float(x)) for x in xs], dtype=np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, (xs[bad[:5]], got[bad[:5]], ref[bad[:5]])
+
+
+def test_e4m3_saturates(oracle_mod):
+    assert oracle_mod.f32_to_e4m3(1e6) == 0x7E and oracle_mod.f32_to_e4m3(-1e6) == 0xFE
+    assert oracle_mod.f32_to_e4m3(479.0) == 0x7E          # rounds to 480 > 448
+    assert oracle_mod.f32_to_e4m3(float("inf")) == 0x7E
+
+
+def test_e8m0_is_a_power_of_two(oracle_mod):
+    for c in (0, 1, 100, 127, 128, 254):
+        assert oracle_mod.e8m0_decode(c) == 2.0 ** (c - 127)
+
+
+# ---------------------------------------------------------- block quant --
+
+@pytest.mark.parametrize("kind", [NVFP4, MXFP4])
+def test_bits_per_weight_from_buffer_sizes(oracle_mod, kind):
+    fx = golden("fp4_formats.json")
+    N, K = 8, 256
+    codes, scales = oracle_mod.fp4_quant(bf16(np.ones((N, K), np.float32)), kind)
+    bits = (codes.nbytes + scales.nbytes) * 8 / (N * K)
+    if kind == NVFP4:
+        assert bits == fx["nvfp4"]["bits_per_weight"]               # printed on page 2
+    else:
+        assert bits == 4 + fx["mxfp4"]["scale_bits"] / fx["mxfp4"]["block"]
+
+
+@pytest.mark.parametrize("kind", [NVFP4, MXFP4])
+@pytest.mark.parametrize("sigma", [1.0, 0.02])
+def test_block_quant_follows_definition(oracle_mod, kind, sigma):
+    """Every scale and every code against the definitions, computed here in
+    exact arithmetic: the scale from the block's amax (E4M3 of fl32(amax/6) by
+    torch's conversion for NVFP4; 2^(floor(log2 amax) - 2) for MXFP4) and each
+    code as the nearest E2M1 value of fl32(w / scale), ties to even, saturated."""
+    rng = np.random.default_rng(11 + kind)
+    N, K = 6, 128
+    Wb = bf16((rng.standard_normal((N, K)) * sigma).astype(np.float32))
+    W = bf16_value(Wb)
+    codes, scales = oracle_mod.fp4_quant(Wb, kind)
+    B = 16 if kind == NVFP4 else 32
+    for n in range(N):
+        for b in range(K // B):
+            blk = W[n, b * B:(b + 1) * B]
+            amax = float(np.max(np.abs(blk)))
+            if kind == NVFP4:
+                t = np.float32(np.float32(amax) / np.float32(6.0))
+                sc_ref = int(torch.tensor([t]).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+                s = float(torch.tensor([sc_ref], dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).float()[0])
+            else:
+                e = max(-127, min(127, int(np.floor(np.log2(amax))) - 2)) if amax > 0 else -127
+                sc_ref, s = e + 127, 2.0 ** e
+            assert scales[n, b] == sc_ref, (n, b)
+            for i in range(B):
+                k = b * B + i
+                q = (codes[n, k // 2] >> (4 * (k & 1))) & 15
+                want = 0.0 if s == 0 else e2m1_nearest(float(np.float32(np.float32(blk[i]) / np.float32(s))))
+                assert oracle_mod.e2m1_decode(q) == want, (n, k, blk[i], s)
+
+
+def test_nvfp4_block_maximum_maps_to_six(oracle_mod):
+    """With a normal E4M3 scale, amax / s lies within 6 (1 -+ 2^-4)^-1, which
+    rounds (or saturates) to 6: every block holds a code of magnitude 6."""
+    rng = np.random.default_rng(21)
+    Wb = bf16((rng.standard_normal((16, 256)) * 2.0).astype(np.float32))
+    codes, scales = oracle_mod.fp4_quant(Wb, NVFP4)
+    vals = oracle_mod.fp4_dequant(codes, scales, NVFP4)
+    for n in range(16):
+        for b in range(16):
+            s = oracle_mod.e4m3_decode(int(scales[n, b]))
+            assert s >= golden("fp4_formats.json")["e4m3"]["min_normal"]
+            assert np.max(np.abs(vals[n, b * 16:(b + 1) * 16])) == 6.0 * s
+
+
+def test_mxfp4_block_maximum_maps_to_four_or_six(oracle_mod):
+    """amax / 2^(floor(log2 amax) - 2) lies in [4, 8): the block maximum's code
+    is 4 or 6 (values of 7 and above saturate to 6)."""
+    rng = np.random.default_rng(22)
+    Wb = bf16((rng.standard_normal((16, 256)) * 0.02).astype(np.float32))
+    codes, scales = oracle_mod.fp4_quant(Wb, MXFP4)
+    W = bf16_value(Wb)
+    for n in range(16):
+        for b in range(8):
+            s = oracle_mod.e8m0_decode(int(scales[n, b]))
+            r = np.max(np.abs(W[n, b * 32:(b + 1) * 32])) / s
+            assert 4.0 <= r < 8.0
+            q = [(codes[n, k // 2] >> (4 * (k & 1))) & 15 for k in range(b * 32, (b + 1) * 32)]
+            assert max(abs(oracle_mod.e2m1_decode(c)) for c in q) in (4.0, 6.0)
+
+
+@pytest.mark.parametrize("kind", [NVFP4, MXFP4])
+def test_dequant_is_the_exact_product_and_fits_bf16(oracle_mod, kind):
+    rng = np.random.default_rng(23)
+    Wb = bf16((rng.standard_normal((4, 64)) * 0.5).astype(np.float32))
+    codes, scales = oracle_mod.fp4_quant(Wb, kind)
+    got = oracle_mod.fp4_dequant(codes, scales, kind)
+    B = 16 if kind == NVFP4 else 32
+    for n in range(4):
+        for k in range(64):
+            q = (codes[n, k // 2] >> (4 * (k & 1))) & 15
+            sc = int(scales[n, k // B])
+            s = oracle_mod.e4m3_decode(sc) if kind == NVFP4 else oracle_mod.e8m0_decode(sc)
+            assert float(got[n, k]) == oracle_mod.e2m1_decode(q) * s
+    assert np.array_equal(bf16_value(bf16(got)), got)
+
+
+def test_packing_puts_the_even_element_in_the_low_nibble(oracle_mod):
+    # a 16-weight block with amax 3: s = e4m3(0.5) = 0.5, so w = 3 -> 6 (code 0b0111) and
+    # w = -1 -> -2 (code 0b1100)
+    w = np.zeros((1, 16), np.float32)
+    w[0, 0], w[0, 1], w[0, 2] = 3.0, -1.0, 0.5
+    codes, scales = oracle_mod.fp4_quant(bf16(w), NVFP4)
+    assert oracle_mod.e4m3_decode(int(scales[0, 0])) == 0.5
+    assert codes[0, 0] == (0xC << 4) | 0x7          # element 0 low nibble, element 1 high nibble
+    assert codes[0, 1] == 0x2                       # element 2 = 0.5 / 0.5 = 1.0 -> code 2
+
+
+def test_zero_block_gives_zero_codes(oracle_mod):
+    for kind in (NVFP4, MXFP4):
+        codes, scales = oracle_mod.fp4_quant(np.zeros((2, 64), np.uint16), kind)
+        assert not codes.any()
+        assert np.all(oracle_mod.fp4_dequant(codes, scales, kind) == 0.0)
