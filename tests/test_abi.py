@@ -106,6 +106,18 @@ def test_gemm_rejects_bad_arguments(w4):
     assert mm(w4, Y=FAKE + 1) == E
 
 
+def test_gemm_rejects_a_missing_or_short_split_k_workspace(w4):
+    """Skinny tensor-core shapes split K and need the caller's workspace: a
+    missing, short or misaligned one is rejected before anything launches."""
+    E = w4.W4_ERR_INVALID_ARG
+    for M, N, K in ((32, 512, 4096), (24, 256, 4096), (17, 130, 2048)):
+        need = w4.w4a16_workspace_bytes(M, N, K, 128)
+        assert need > 0
+        assert mm(w4, M=M, N=N, K=K) == E                                  # no workspace
+        assert mm(w4, M=M, N=N, K=K, ws=FAKE, wsb=need - 1) == E           # one byte short
+        assert mm(w4, M=M, N=N, K=K, ws=FAKE + 64, wsb=need) == E          # not 256-byte aligned
+
+
 def test_workspace_query_is_host_only(w4):
     for M in (1, 4, 8, 16, 32, 512, 8192):
         assert w4.w4a16_workspace_bytes(M, 4096, 4096, 128) >= 0
