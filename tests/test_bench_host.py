@@ -57,3 +57,30 @@ def test_max_over_ranks_gloo():
         assert p.exitcode == 0
     for rank, ms, units in res:
         assert ms == 15.0 and units == 300.0
+
+
+@pytest.mark.parametrize("workload", ["decode", "awq"])
+def test_reference_arm_prints_one_complete_line(workload):
+    """`bench.py --impl reference` (the CPU oracle on a bounded sample) prints
+    one JSON line with the base contract's keys and the same workload
+    description as the library's arm."""
+    import json
+    import subprocess
+    import sys
+    out = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"), "--impl",
+                          "reference", "--workload", workload, "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["value"] > 0 and d["warmup"] >= 3
+    assert d["unit"] == "GB/s" and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    want = (bench.WORKLOAD_DESC[workload] if workload != "awq" else
+            bench.awq_desc(bench.AWQ_SHAPE["M"], bench.AWQ_SHAPE["N"], bench.AWQ_SHAPE["K"],
+                           bench.AWQ_SHAPE["group"], bench.AWQ_SHAPE["n_alpha"]))
+    assert d["config"]["workload"] == want
