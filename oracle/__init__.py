@@ -280,3 +280,11 @@ def fp4_dequant(codes: np.ndarray, scales: np.ndarray, kind: int) -> np.ndarray:
     if lib().orc_fp4_dequant_rows(_ptr(codes), _ptr(scales), N, K, kind, _ptr(out)) != 0:
         raise ValueError("K must be a multiple of the block")
     return out
+
+
+def fp4_reference(X_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, kind: int, threads: int = 1) -> np.ndarray:
+    """Y[m][n] = sum_k x[m][k] * w^[n][k] in fp64 with the FP4-dequantized weights
+    (X bf16 [M, K]).  w^ is exact in bf16, so this is gemm_f64 of its bf16 bits."""
+    What = fp4_dequant(codes, scales, kind)
+    What_bits = (What.view(np.uint32) >> 16).astype(np.uint16)
+    return gemm_f64(X_bits, What_bits, threads=threads)

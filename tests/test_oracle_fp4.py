@@ -208,3 +208,36 @@ def test_zero_block_gives_zero_codes(oracle_mod):
         codes, scales = oracle_mod.fp4_quant(np.zeros((2, 64), np.uint16), kind)
         assert not codes.any()
         assert np.all(oracle_mod.fp4_dequant(codes, scales, kind) == 0.0)
+
+
+@pytest.mark.parametrize("kind", [NVFP4, MXFP4])
+def test_product_reference_selects_dequantized_columns(oracle_mod, kind):
+    """One-hot activation rows pick columns of w^ (the product's orientation),
+    and a dense product equals a plain fp64 matrix product of the decoded
+    weights (decoded here from the codes and scales, not by the oracle)."""
+    rng = np.random.default_rng(31 + kind)
+    N, K = 12, 64
+    Wb = bf16((rng.standard_normal((N, K)) * 0.5).astype(np.float32))
+    codes, scales = oracle_mod.fp4_quant(Wb, kind)
+    B = 16 if kind == NVFP4 else 32
+    Wd = np.zeros((N, K))
+    for n in range(N):
+        for k in range(K):
+            q = int((codes[n, k // 2] >> (4 * (k & 1))) & 15)
+            mag = E2M1_VALUES[q & 7] * (-1.0 if q & 8 else 1.0)
+            sc = int(scales[n, k // B])
+            if kind == NVFP4:
+                s = float(torch.tensor([sc], dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).float()[0])
+            else:
+                s = 2.0 ** (sc - 127)
+            Wd[n, k] = mag * s
+    ks = [0, 17, 63]
+    X = np.zeros((len(ks), K), np.float32)
+    for m, k in enumerate(ks):
+        X[m, k] = 1.0
+    Y = oracle_mod.fp4_reference(bf16(X), codes, scales, kind)
+    for m, k in enumerate(ks):
+        assert np.array_equal(Y[m], Wd[:, k])
+    Xr = bf16((rng.standard_normal((5, K))).astype(np.float32))
+    Y = oracle_mod.fp4_reference(Xr, codes, scales, kind)
+    assert np.allclose(Y, bf16_value(Xr).astype(np.float64) @ Wd.T, rtol=1e-12, atol=1e-12)
