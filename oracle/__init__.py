@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.orc_fp4_quant_rows.restype = I
         L.orc_fp4_dequant_rows.argtypes = [P, P, I64, I64, I, P]
         L.orc_fp4_dequant_rows.restype = I
+        L.orc_mxfp8_quant_rows.argtypes = [P, I64, I64, P, P]
+        L.orc_mxfp8_quant_rows.restype = I
+        L.orc_mxfp8_dequant_rows.argtypes = [P, P, I64, I64, P]
+        L.orc_mxfp8_dequant_rows.restype = I
         _lib = L
     return _lib
 
@@ -288,3 +292,35 @@ def fp4_reference(X_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, kin
     What = fp4_dequant(codes, scales, kind)
     What_bits = (What.view(np.uint32) >> 16).astype(np.uint16)
     return gemm_f64(X_bits, What_bits, threads=threads)
+
+
+def mxfp8_quant(X_bits: np.ndarray):
+    """MXFP8 activations (page 3 section 4.3: activations kept at FP8, MX blocks
+    of 32 with an E8M0 scale): returns (codes uint8 [M, K] E4M3, scales uint8
+    [M, K/32] E8M0).  The scale rule is stated in w4_oracle.c."""
+    X_bits = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    M, K = X_bits.shape
+    codes = np.zeros((M, K), dtype=np.uint8)
+    scales = np.zeros((M, K // 32), dtype=np.uint8)
+    if lib().orc_mxfp8_quant_rows(_ptr(X_bits), M, K, _ptr(codes), _ptr(scales)) != 0:
+        raise ValueError("K must be a multiple of 32")
+    return codes, scales
+
+
+def mxfp8_dequant(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """x^ = e4m3(code) * scale as fp32 [M, K] (exact)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    M, K = codes.shape
+    out = np.zeros((M, K), dtype=np.float32)
+    if lib().orc_mxfp8_dequant_rows(_ptr(codes), _ptr(scales), M, K, _ptr(out)) != 0:
+        raise ValueError("K must be a multiple of 32")
+    return out
+
+
+def mx_reference(x_codes, x_scales, w_codes, w_scales) -> np.ndarray:
+    """Y[m][n] = sum_k x^[m][k] * w^[n][k] in fp64 for MXFP8 activations and
+    MXFP4 weights (both factors exact in fp32)."""
+    Xd = mxfp8_dequant(x_codes, x_scales).astype(np.float64)
+    Wd = fp4_dequant(w_codes, w_scales, MXFP4).astype(np.float64)
+    return Xd @ Wd.T

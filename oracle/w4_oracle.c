@@ -468,3 +468,51 @@ int orc_fp4_dequant_rows(const uint8_t *codes, const uint8_t *scales, int64_t N,
         }
     return 0;
 }
+
+/* MXFP8 activations for the block-scaled tensor-core product (page 3 section
+ * 4.3: FP4 for the weights, activations kept at FP8; MX blocks of 32 share an
+ * E8M0 scale).  Reading: the OCP Microscaling rule with the E4M3 maximum
+ * exponent 8 (448 = 1.75 * 2^8): scale 2^(floor(log2 amax) - 8) clamped to
+ * [-127, 127], elements e4m3_rn(fl32(x / scale)) saturating at 448; an
+ * all-zero block gets 2^-127 and zero codes.  X: bf16 [M, K]; codes: uint8
+ * [M, K] (E4M3); scales: uint8 [M, K/32] (E8M0). */
+int orc_mxfp8_quant_rows(const uint16_t *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales)
+{
+    if (K % 32 != 0) return -1;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const uint16_t *x = X + m * K + b * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(orc_bf16_to_f32(x[i]));
+                if (a > amax) amax = a;
+            }
+            int e = -127;
+            if (amax > 0.0f) {
+                int ex;
+                frexp((double)amax, &ex);
+                e = (ex - 1) - 8;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            scales[m * (K / 32) + b] = (uint8_t)(e + 127);
+            const float sc = orc_e8m0_decode(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                volatile float t = orc_bf16_to_f32(x[i]) / sc;      /* one IEEE division */
+                codes[m * K + b * 32 + i] = (uint8_t)orc_f32_to_e4m3_sat(t);
+            }
+        }
+    }
+    return 0;
+}
+
+/* x^[m][k] = e4m3(code) * scale, fp32 [M, K] (exact). */
+int orc_mxfp8_dequant_rows(const uint8_t *codes, const uint8_t *scales, int64_t M, int64_t K, float *out)
+{
+    if (K % 32 != 0) return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k)
+            out[m * K + k] = (float)((double)orc_e4m3_decode(codes[m * K + k]) *
+                                     (double)orc_e8m0_decode(scales[m * (K / 32) + k / 32]));
+    return 0;
+}

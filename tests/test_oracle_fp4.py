@@ -241,3 +241,69 @@ def test_product_reference_selects_dequantized_columns(oracle_mod, kind):
     Xr = bf16((rng.standard_normal((5, K))).astype(np.float32))
     Y = oracle_mod.fp4_reference(Xr, codes, scales, kind)
     assert np.allclose(Y, bf16_value(Xr).astype(np.float64) @ Wd.T, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------- MXFP8 activations --
+
+def _e4m3_code_torch(t: float) -> int:
+    """torch's E4M3 code of t after saturation to +-448 (torch's own conversion
+    gives NaN above the range; rounding never takes a value <= 448 above it)."""
+    t = max(-448.0, min(448.0, t))
+    return int(torch.tensor([t], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+
+
+@pytest.mark.parametrize("sigma", [1.0, 40.0, 1e-3])
+def test_mxfp8_follows_definition(oracle_mod, sigma):
+    """Scale 2^(floor(log2 amax) - 8) per 32 activations, codes E4M3 of
+    fl32(x / scale) saturated at 448 (torch's conversion), checked one by one."""
+    rng = np.random.default_rng(41)
+    M, K = 4, 128
+    Xb = bf16((rng.standard_normal((M, K)) * sigma).astype(np.float32))
+    X = bf16_value(Xb)
+    codes, scales = oracle_mod.mxfp8_quant(Xb)
+    for m in range(M):
+        for b in range(K // 32):
+            blk = X[m, b * 32:(b + 1) * 32]
+            amax = float(np.max(np.abs(blk)))
+            e = max(-127, min(127, int(np.floor(np.log2(amax))) - 8)) if amax > 0 else -127
+            assert scales[m, b] == e + 127
+            for i in range(32):
+                t = float(np.float32(np.float32(blk[i]) / np.float32(2.0 ** e)))
+                assert codes[m, b * 32 + i] == _e4m3_code_torch(t), (m, b, i)
+
+
+def test_mxfp8_block_maximum_and_exact_dequant(oracle_mod):
+    """amax / scale lies in [256, 512): the block maximum's code is at least
+    256 (448 when saturated), and x^ = e4m3(code) * scale exactly."""
+    rng = np.random.default_rng(42)
+    Xb = bf16((rng.standard_normal((8, 256)) * 3.0).astype(np.float32))
+    codes, scales = oracle_mod.mxfp8_quant(Xb)
+    d = oracle_mod.mxfp8_dequant(codes, scales)
+    for m in range(8):
+        for b in range(8):
+            s = oracle_mod.e8m0_decode(int(scales[m, b]))
+            vals = [oracle_mod.e4m3_decode(int(c)) for c in codes[m, b * 32:(b + 1) * 32]]
+            assert 256.0 <= max(abs(v) for v in vals) <= 448.0
+            assert all(float(d[m, b * 32 + i]) == vals[i] * s for i in range(32))
+
+
+def test_mx_product_reference(oracle_mod):
+    """One-hot activation rows are exact in MXFP8 (1.0 = 256 * 2^-8) and pick
+    columns of w^; a dense product equals the fp64 product of the two
+    dequantized operands."""
+    rng = np.random.default_rng(43)
+    N, K = 10, 96
+    Wb = bf16((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+    wc, ws = oracle_mod.fp4_quant(Wb, MXFP4)
+    Wd = oracle_mod.fp4_dequant(wc, ws, MXFP4).astype(np.float64)
+    ks = [3, 40, 95]
+    X = np.zeros((len(ks), K), np.float32)
+    for m, k in enumerate(ks):
+        X[m, k] = 1.0
+    xc, xs = oracle_mod.mxfp8_quant(bf16(X))
+    Y = oracle_mod.mx_reference(xc, xs, wc, ws)
+    for m, k in enumerate(ks):
+        assert np.array_equal(Y[m], Wd[:, k])
+    xc, xs = oracle_mod.mxfp8_quant(bf16((rng.standard_normal((6, K))).astype(np.float32)))
+    Xd = oracle_mod.mxfp8_dequant(xc, xs).astype(np.float64)
+    assert np.allclose(oracle_mod.mx_reference(xc, xs, wc, ws), Xd @ Wd.T, rtol=1e-12, atol=1e-15)
