@@ -14,6 +14,8 @@ import ctypes
 import os
 
 SYM, ASYM = 0, 1
+NVFP4, MXFP4 = 0, 1
+FP4_BLOCK = {NVFP4: 16, MXFP4: 32}
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
@@ -46,6 +48,8 @@ def lib() -> ctypes.CDLL:
         L.w4_awq_workspace_bytes.restype = SZ
         L.w4_awq_search.argtypes = [P, P, I64, I64, I64, I, I, I, P, P, P, P, SZ, P]
         L.w4_awq_search.restype = I
+        L.w4_fp4_quant.argtypes = [P, I64, I64, I, P, P, P]
+        L.w4_fp4_quant.restype = I
         L.w4_status_string.argtypes = [I]
         L.w4_status_string.restype = ctypes.c_char_p
         L.w4_layout_version.argtypes = []
@@ -83,6 +87,10 @@ def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, wor
                   stream) -> int:
     return lib().w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, workspace,
                                workspace_bytes, stream)
+
+
+def w4_fp4_quant(W, N, K, kind, codes, scales, stream) -> int:
+    return lib().w4_fp4_quant(W, N, K, kind, codes, scales, stream)
 
 
 def w4_status_string(status: int) -> str:
@@ -188,3 +196,20 @@ def awq_search(W, X, group: int = 128, mode: int = SYM, n_alpha: int = 20, strea
     if st != W4_OK:
         raise W4Error(st, "w4_awq_search")
     return losses, best, s_best
+
+
+def fp4_quant(W, kind: int = NVFP4, stream=None, out=None):
+    """Block-scaled FP4 quantization of a bf16 CUDA tensor W[N,K].
+    Returns (codes uint8 [N, K/2], scales uint8 [N, K/block])."""
+    import torch
+    N, K = W.shape
+    B = FP4_BLOCK.get(kind, 16)
+    if out is None:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+        scales = torch.empty((N, max(K // B, 1)), dtype=torch.uint8, device=W.device)
+    else:
+        codes, scales = out
+    st = w4_fp4_quant(_ptr(W), N, K, kind, _ptr(codes), _ptr(scales), _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_fp4_quant")
+    return codes, scales

@@ -50,6 +50,18 @@ w4_status w4_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
+                       w4_stream_t stream)
+{
+    if (!W || !codes || !scales) return W4_ERR_INVALID_ARG;
+    if (kind != W4_NVFP4 && kind != W4_MXFP4) return W4_ERR_INVALID_ARG;
+    const int64_t B = kind == W4_NVFP4 ? 16 : 32;
+    if (N < 1 || K < B || K % B != 0 || !fits(N, K)) return W4_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(codes, 16)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e = w4::launch_fp4_quant(W, N, K, kind, codes, scales, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group)
 {
     (void)group;

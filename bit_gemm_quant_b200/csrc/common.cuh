@@ -66,6 +66,8 @@ cudaError_t launch_quant_pack(const void *W, int64_t N, int64_t K, int group, in
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                         const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                         cudaStream_t stream);
+cudaError_t launch_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
+                             cudaStream_t stream);
 size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
 // byte range of the split-K tile counters inside that workspace (0 bytes if none)
 void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size_t *bytes);

@@ -78,6 +78,9 @@ typedef enum {
 
 typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
 
+/* Block-scaled FP4 kinds for w4_fp4_quant. */
+typedef enum { W4_NVFP4 = 0, W4_MXFP4 = 1 } w4_fp4_kind;
+
 /*
  * w4_quant_pack -- fold, group-quantize and pack a bf16 weight matrix.
  *   (page 5 section 2.2 formulas; page 2 group quantization; page 3 sections
@@ -186,6 +189,35 @@ w4_status w4_awq_search(const void *W, const void *X, int64_t N, int64_t K, int6
 w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                              const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                              w4_stream_t stream);
+
+/*
+ * w4_fp4_quant -- block-scaled FP4 quantization of a bf16 weight matrix.
+ *   (page 2, the Blackwell FP4 paragraph: E2M1 values, blocks of 16 sharing an
+ *    FP8 E4M3 scale with amax mapped to 6; page 3 section 4.3: MXFP4, blocks of
+ *    32 sharing an E8M0 scale, two FP4 values per byte; page 5 section 2.1:
+ *    the E2M1 set {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6} and E4M3)
+ *   Exact semantics, per block of B consecutive weights of a row:
+ *     amax = max |w| over the block
+ *     W4_NVFP4 (B = 16): scale code = e4m3_rne_satfinite(fl32(amax / 6));
+ *                        s = its value (0 when it rounds to 0)
+ *     W4_MXFP4 (B = 32): e = clamp(floor(log2 amax) - 2, -127, 127) (-127 for
+ *                        an all-zero block); scale code = e + 127 (E8M0); s = 2^e
+ *     code = e2m1_rne_satfinite(fl32(w / s)) for s > 0, else 0: the nearest
+ *            E2M1 value, ties to the even fraction bit, magnitudes above 6
+ *            giving 6; the sign bit is w / s's sign bit
+ *     w^   = e2m1(code) * s (exact; the pages' snippet multiplies by 6.0 a
+ *            second time, which would map amax to 36, and is not followed)
+ *   W        bf16 [N][K], finite, 16-byte aligned (codes of a block holding
+ *            an infinity or NaN are unspecified).
+ *   N, K     N >= 1, K >= B, K % B == 0.
+ *   kind     W4_NVFP4 or W4_MXFP4.
+ *   codes    out, uint8 [N][K/2], 16-byte aligned: element 2i of a row in the
+ *            low nibble of byte i, element 2i+1 in the high nibble.
+ *   scales   out, uint8 [N][K/B]: E4M3 codes (NVFP4) or E8M0 codes (MXFP4).
+ * Every output byte is written; outputs must not overlap inputs.
+ */
+w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
+                       w4_stream_t stream);
 
 /* Text for a status code; never NULL. */
 const char *w4_status_string(int status);
