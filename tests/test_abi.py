@@ -31,7 +31,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("w4_quant_pack", "w4a16_gemm", "w4a16_workspace_bytes", "w4_status_string",
-              "w4_layout_version", "w4_device_error"):
+              "w4_layout_version", "w4_device_error", "w4_fp4_quant"):
         assert n in names
 
 
@@ -116,6 +116,27 @@ def test_gemm_rejects_a_missing_or_short_split_k_workspace(w4):
         assert mm(w4, M=M, N=N, K=K) == E                                  # no workspace
         assert mm(w4, M=M, N=N, K=K, ws=FAKE, wsb=need - 1) == E           # one byte short
         assert mm(w4, M=M, N=N, K=K, ws=FAKE + 64, wsb=need) == E          # not 256-byte aligned
+
+
+def fq(w4, W=FAKE, N=4, K=64, kind=0, c=FAKE, sc=FAKE):
+    return w4.w4_fp4_quant(P(W) if W else None, N, K, kind, P(c) if c else None, P(sc) if sc else None, None)
+
+
+def test_fp4_quant_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    assert fq(w4, W=0) == E
+    assert fq(w4, c=0) == E
+    assert fq(w4, sc=0) == E
+    assert fq(w4, kind=2) == E and fq(w4, kind=-1) == E
+    assert fq(w4, N=0) == E                      # empty input
+    assert fq(w4, K=0) == E
+    assert fq(w4, K=8) == E                      # shorter than an NVFP4 block
+    assert fq(w4, K=48, kind=1) == E             # not a whole number of MXFP4 blocks
+    assert fq(w4, K=16, kind=1) == E
+    assert fq(w4, K=40, kind=0) == E
+    assert fq(w4, W=FAKE + 2) == E               # uint4 loads need 16-byte alignment
+    assert fq(w4, c=FAKE + 8) == E
+    assert fq(w4, N=1 << 40, K=1 << 30) == E     # N*K overflows int64
 
 
 def test_workspace_query_is_host_only(w4):
