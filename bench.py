@@ -13,6 +13,8 @@ every activation batch is multiplied by its packed weight (w4a16_gemm).
   prefill           K=4096, N=14336, asymmetric g=128: 1 x w4_quant_pack + M in {512,2048,8192};
                     value = GEMM TFLOP/s over the step
   quantizer         W[28672, 8192]: g in {32,64,128} x {sym, asym} + smoothing fold
+  awq               the AWQ scale search over W[4096, 4096] with 128 calibration rows
+  fp4quant          W[28672, 8192] to NVFP4 and to MXFP4: 2 x w4_fp4_quant per step
 
 The K timed steps are captured in one CUDA graph (kernel nodes only) and
 replayed once between CUDA events on the launching stream.  Inputs rotate over
@@ -52,7 +54,8 @@ if ROOT not in sys.path:
 from bit_gemm_quant_b200 import roofline, synth  # noqa: E402
 
 METRIC = "W4A16 g128 GEMV HBM GB/s (% peak); GEMM TFLOPS (% peak); quant-pack GB/s"
-KERNEL_SOURCES = {"w4_quant_pack": "quant_pack.cu", "w4a16_gemv": "gemv.cu", "w4a16_gemm_tc": "gemm_tc.cu"}
+KERNEL_SOURCES = {"w4_quant_pack": "quant_pack.cu", "w4a16_gemv": "gemv.cu", "w4a16_gemm_tc": "gemm_tc.cu",
+                  "w4_fp4_quant": "fp4_quant.cu"}
 THROTTLE_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -62,7 +65,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["w4", "reference"], default="w4")
-    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "awq"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "awq", "fp4quant"], default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -115,6 +118,8 @@ WORKLOAD_DESC = {
     "smallbatch": "small-batch decode: K=8192, N=28672, symmetric INT4 g=128, M in {2,4,8,16,32}; step = 1 w4_quant_pack + 5 w4a16_gemm",
     "prefill": "prefill GEMM: K=4096, N=14336, asymmetric INT4 g=128, M in {512,2048,8192}; step = 1 w4_quant_pack + 3 w4a16_gemm",
     "quantizer": "quantizer sweep: W[28672,8192], g in {32,64,128} x {sym,asym} + smoothing fold; step = 7 w4_quant_pack",
+    "fp4quant": "block-scaled FP4 weight quantization: W[28672,8192] bf16 to NVFP4 (E2M1, E4M3 scale per 16) and "
+                "to MXFP4 (E2M1, E8M0 scale per 32); step = 2 w4_fp4_quant",
 }
 
 
@@ -607,6 +612,8 @@ def run_reference(args, rank, world):
     oracle.build()
     if args.workload == "awq":
         return run_reference_awq(args, world)
+    if args.workload == "fp4quant":
+        return run_reference_fp4(args, world)
     plist = problems_for(args.workload)
     keys = list(dict.fromkeys(k for k, _ in plist))
     first = {k: p for k, p in reversed(plist)}
@@ -663,6 +670,24 @@ def run_reference_awq(args, world):
     sample = ("the search over %d output channels per step (rotating), all %d calibration rows and %d alphas: "
               "oracle fold+quantize+pack, dequantize, fp64 products and losses, single thread" % (rows, M, na))
     print_reference(args, world, val, "GB/s", dt * 1e3 / args.steps, awq_desc(M, N, K, g, na), sample)
+
+
+def run_reference_fp4(args, world):
+    """The oracle's NVFP4 and MXFP4 quantizers on `rows` rows of the bench's
+    weight per step (rotating), single thread."""
+    import oracle
+    N, K = FP4_SHAPE["N"], FP4_SHAPE["K"]
+    rows = 16
+    W = fp4_weight(0)
+    for si in range(max(3, args.warmup)):
+        oracle_fp4_sample(oracle, W, rows, si * rows)
+    nb = 0
+    t0 = time.perf_counter()
+    for si in range(args.steps):
+        nb += oracle_fp4_sample(oracle, W, rows, si * rows)
+    dt = time.perf_counter() - t0
+    sample = "%d rows of W[%d,%d] per step (rotating), NVFP4 and MXFP4, oracle, single thread" % (rows, N, K)
+    print_reference(args, world, nb / dt / 1e9, "GB/s", dt * 1e3 / args.steps, WORKLOAD_DESC["fp4quant"], sample)
 
 
 # ------------------------------------------------------------ awq search --
@@ -768,6 +793,224 @@ def run_awq(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------- FP4 quantization --
+
+FP4_SHAPE = dict(N=28672, K=8192)
+FP4_KINDS = (("nvfp4", 0, 16), ("mxfp4", 1, 32))
+
+
+def fp4_weight(rank_seed: int) -> np.ndarray:
+    """The quantizer sweep's weight: W[28672, 8192] ~ N(0, 0.02^2), bf16 bits."""
+    return synth.weights(4 + rank_seed, FP4_SHAPE["N"], FP4_SHAPE["K"], 0.02)
+
+
+def fp4_step_bytes() -> int:
+    N, K = FP4_SHAPE["N"], FP4_SHAPE["K"]
+    return sum(roofline.fp4_quant_bytes(N, K, B) for _, _, B in FP4_KINDS)
+
+
+def oracle_fp4_sample(oracle, W, rows: int, offset: int) -> int:
+    """Both oracle quantizers on rows [offset, offset + rows) of W; returns the
+    algorithmic bytes processed."""
+    N, K = W.shape
+    r0 = offset % N
+    r1 = min(N, r0 + rows)
+    nb = 0
+    for _, kind, B in FP4_KINDS:
+        oracle.fp4_quant(W[r0:r1], kind)
+        nb += roofline.fp4_quant_bytes(r1 - r0, K, B)
+    return nb
+
+
+def run_fp4(args, rank, world, local_rank):
+    """Block-scaled FP4 weight quantization of the quantizer sweep's weight
+    (W[28672, 8192], 470 MB, larger than L2, so every launch reads it from
+    HBM): one step is its NVFP4 and its MXFP4 quantization."""
+    import torch
+    import bit_gemm_quant_b200 as w4
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    w4.lib()
+    pk = roofline.peaks(ROOT)
+    N, K = FP4_SHAPE["N"], FP4_SHAPE["K"]
+    host_W = fp4_weight(1000 * rank)
+    W = torch.from_numpy(host_W.view(np.int16)).to(device).view(torch.bfloat16)
+    outs = {name: w4.fp4_quant(W, kind) for name, kind, _ in FP4_KINDS}
+
+    def step():
+        for name, kind, _ in FP4_KINDS:
+            w4.fp4_quant(W, kind, out=outs[name])
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    K_steps = args.steps
+    graph = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(device)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cs):
+        for _ in range(K_steps):
+            step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(smi_gpu_id(local_rank))
+    sampler.start()
+    sampler.mark_begin()
+    t_end = time.time() + 1.5
+    replays = 0
+    while time.time() < t_end or replays < 2:
+        graph.replay()
+        replays += 1
+        torch.cuda.synchronize()
+
+    def timed():
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(cs):
+            e0.record(cs)
+            graph.replay()
+            e1.record(cs)
+        e1.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
+
+    local_ms = timed()
+    sampler.mark_end()
+    clocks = sampler.stop()
+    if any(r in clocks.get("reasons", []) for r in THROTTLE_REASONS):
+        sampler = ClockSampler(sampler.gpu_id)
+        sampler.start()
+        sampler.mark_begin()
+        local_ms = timed()
+        sampler.mark_end()
+        clocks = sampler.stop()
+        clocks["remeasured"] = True
+    del graph
+
+    # each kind alone: a graph of KL launches between CUDA events on its stream,
+    # median and min over 5 replays (W is 470 MB, so every launch reads it from HBM)
+    KL = max(K_steps, 20)
+    kernels = {}
+    for name, kind, B in FP4_KINDS:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            for _ in range(KL):
+                w4.fp4_quant(W, kind, out=outs[name])
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        per = []
+        for _ in range(5):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(cs):
+                e0.record(cs)
+                g.replay()
+                e1.record(cs)
+            e1.synchronize()
+            per.append(e0.elapsed_time(e1) / KL)
+        del g
+        avg, mn = statistics.median(per), min(per)
+        nbytes = roofline.fp4_quant_bytes(N, K, B)
+        kernels["w4_fp4_quant[%s]" % name] = {
+            "launches": KL * 5, "avg_us": round(avg * 1e3, 3), "min_us": round(mn * 1e3, 3), "bytes": nbytes,
+            "gbs": round(nbytes / (avg * 1e-3) / 1e9, 1),
+            "hbm_frac": round(nbytes / (avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+
+    work = K_steps * fp4_step_bytes()
+    max_ms, total = aggregate(local_ms, work, device)
+    value = total / (max_ms * 1e-3) / 1e9
+    # the roofline entry is the kernel over both kinds: bytes per launch averaged
+    # over the two launches of a step, divided by their average duration
+    tot_us = sum(v["avg_us"] for v in kernels.values())
+    per_launch = fp4_step_bytes() / len(FP4_KINDS)
+    achieved = per_launch / (tot_us * 1e-6 / len(FP4_KINDS)) / 1e9
+    traffic = traffic_table()
+    tr = [traffic.get(("w4_fp4_quant", name)) for name, _, _ in FP4_KINDS]
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4),
+            "traffic": (sum(tr) / len(tr)) if all(t is not None for t in tr) else None,
+            "kernel": "w4_fp4_quant", "algorithmic_per_launch": per_launch,
+            "peak_source": "%s (%s)" % (pk["source"], "MEASURED_PEAKS.json" if pk["source"] == "measured"
+                                        else "recipe")}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = fp4_e2e(w4, torch, device, host_W, min(K_steps, 5))
+        e_ms, e_work = aggregate(e2e["ms"], e2e["work"], device)
+        e2e = {"value": round(e_work / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        t0 = time.perf_counter()
+        oracle_fp4_sample(oracle, host_W, 16, 0)
+        dt = time.perf_counter() - t0
+        rows = min(N, max(16, int(16 * args.cpu_budget / max(dt, 1e-3))))
+        t0 = time.perf_counter()
+        nb = oracle_fp4_sample(oracle, host_W, rows, 0)
+        dt = time.perf_counter() - t0
+        cpu = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
+               "sample": "first %d rows of W[%d,%d], NVFP4 and MXFP4, oracle, single thread" % (rows, N, K)}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K_steps,
+            "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / K_steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD_DESC["fp4quant"],
+                       "l2": "the 470 MB weight is larger than L2; every launch reads it from HBM",
+                       "timing": "K steps captured in one CUDA graph, replayed between CUDA events on the launching "
+                                 "stream after %d untimed replays; max over ranks" % replays,
+                       "parallelism": "replicas (dp%d), no data-path collective" % world},
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": K_steps * len(FP4_KINDS) * world, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def fp4_e2e(w4, torch, device, host_W, steps):
+    """Both quantizations through the tensor API from a pinned host weight:
+    the host->device copy of W, the two calls and the device->host copies of
+    the codes and scales, all timed."""
+    hW = torch.from_numpy(host_W.view(np.int16)).pin_memory()
+    N, K = host_W.shape
+    h_out = {name: (torch.empty((N, K // 2), dtype=torch.uint8).pin_memory(),
+                    torch.empty((N, K // B), dtype=torch.uint8).pin_memory()) for name, _, B in FP4_KINDS}
+    d2h = sum(c.numel() + s.numel() for c, s in h_out.values())
+
+    def one():
+        Wd = hW.to(device, non_blocking=True).view(torch.bfloat16)
+        for name, kind, _ in FP4_KINDS:
+            c, s = w4.fp4_quant(Wd, kind)
+            h_out[name][0].copy_(c, non_blocking=True)
+            h_out[name][1].copy_(s, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    e1.synchronize()
+    barrier()
+    return {"ms": e0.elapsed_time(e1), "work": fp4_step_bytes() * steps, "h2d": hW.numel() * 2, "d2h": d2h,
+            "steps": steps}
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
@@ -776,6 +1019,9 @@ def main(argv=None):
         return 0
     if args.workload == "awq":
         run_awq(args, rank, world, local_rank)
+        return 0
+    if args.workload == "fp4quant":
+        run_fp4(args, rank, world, local_rank)
         return 0
     run_w4(args, rank, world, local_rank)
     return 0

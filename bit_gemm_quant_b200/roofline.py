@@ -8,6 +8,8 @@ must read and write once (not DRAM counters):
   w4a16_gemm(M, N, K, g):  read qweight (NK/2), scales, qzeros (asym), X (2MK),
                            write Y (2MN)
   FLOPs of w4a16_gemm:     2 M N K
+  w4_fp4_quant(N, K, B):   read W (2NK), write codes (NK/2) and one scale byte
+                           per block of B (N K/B)
 """
 from __future__ import annotations
 
@@ -31,6 +33,10 @@ def quant_pack_bytes(N: int, K: int, g: int, mode: int, smooth: bool = False) ->
 
 def gemm_bytes(M: int, N: int, K: int, g: int, mode: int) -> int:
     return packed_bytes(N, K, g, mode) + 2 * M * K + 2 * M * N
+
+
+def fp4_quant_bytes(N: int, K: int, block: int) -> int:
+    return 2 * N * K + N * K // 2 + N * (K // block)
 
 
 def gemm_flops(M: int, N: int, K: int) -> int:

@@ -24,6 +24,9 @@ def test_algorithmic_bytes():
     assert roofline.gemm_bytes(1, 4096, 4096, 128, 1) == 8732672
     assert roofline.gemm_flops(2048, 14336, 4096) == 2 * 2048 * 14336 * 4096
     assert roofline.quant_pack_bytes(28672, 8192, 128, 0) == 2 * 28672 * 8192 + 28672 * 4096 + 2 * 28672 * 64
+    # bf16 in, two E2M1 codes per byte, one scale byte per block
+    assert roofline.fp4_quant_bytes(28672, 8192, 16) == 28672 * 8192 * 2 + 28672 * 4096 + 28672 * 512
+    assert roofline.fp4_quant_bytes(1, 32, 32) == 64 + 16 + 1
 
 
 def _free_port():
@@ -59,7 +62,7 @@ def test_max_over_ranks_gloo():
         assert ms == 15.0 and units == 300.0
 
 
-@pytest.mark.parametrize("workload", ["decode", "awq"])
+@pytest.mark.parametrize("workload", ["decode", "awq", "fp4quant"])
 def test_reference_arm_prints_one_complete_line(workload):
     """`bench.py --impl reference` (the CPU oracle on a bounded sample) prints
     one JSON line with the base contract's keys and the same workload
