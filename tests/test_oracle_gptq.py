@@ -1,0 +1,152 @@
+"""Pins of the GPTQ oracle (oracle/gptq.py).
+
+None of these re-types the oracle's update. Each checks it against something
+the mathematics fixes independently:
+  * a diagonal Hessian couples no columns, so GPTQ must reduce to plain
+    round-to-nearest, i.e. to the already pinned ``oracle.quant_pack``;
+  * after columns 0..j-1 are fixed to their grid points, the value GPTQ gives
+    column j must be the least-squares optimum of the remaining columns for the
+    objective (w - w~) H (w - w~)^T, computed here by a direct linear solve
+    of the Hessian blocks (no inverse, no Cholesky factor); at a group's first
+    column the group's scale and zero-point must be those of that optimum;
+  * with one calibration row the Hessian is rank one plus the damping term,
+    and the two-column update has a closed form (Sherman-Morrison) in which
+    the damping lambda = 0.01 trace(X^T X) / K appears explicitly;
+  * every column's grid point is within half a step of the value quantized
+    (unless clipped);
+  * on calibration features with low-rank correlation, GPTQ trades a larger
+    weight error for a much smaller output error (page 5 section 2.5, Scene 4,
+    a qualitative check: its setup is not stated).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import gptq
+from bit_gemm_quant_b200 import synth
+
+SYM, ASYM = 0, 1
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    oracle.build()
+
+
+def bits(a):
+    return synth.to_bf16_bits(np.asarray(a, dtype=np.float32))
+
+
+def f64(b):
+    return synth.bf16_bits_to_f32(b).astype(np.float64)
+
+
+def correlated_calibration(seed, M, K, rank, noise=0.05):
+    rng = np.random.default_rng(seed)
+    Z = rng.standard_normal((M, rank))
+    A = rng.standard_normal((rank, K))
+    return bits(Z @ A + noise * rng.standard_normal((M, K)))
+
+
+@pytest.mark.parametrize("mode", [SYM, ASYM])
+@pytest.mark.parametrize("g", [32, 64])
+def test_diagonal_hessian_reduces_to_round_to_nearest(mode, g):
+    K, N = 128, 9
+    rng = np.random.default_rng(1)
+    W = bits(rng.standard_normal((N, K)) * 0.02)
+    X = bits(np.diag(rng.uniform(0.5, 3.0, K)))        # orthogonal columns: X^T X diagonal
+    q, s, z = gptq.gptq_pack(W, X, g, mode)
+    rq, rs, rz = oracle.quant_pack(W, g, mode)
+    assert np.array_equal(q, rq) and np.array_equal(s, rs)
+    if mode == ASYM:
+        assert np.array_equal(z, rz)
+    else:
+        assert z is None and rz is None
+
+
+@pytest.mark.parametrize("mode", [SYM, ASYM])
+def test_each_column_is_the_least_squares_optimum_given_the_fixed_ones(mode):
+    N, K, M, g = 4, 24, 40, 8
+    rng = np.random.default_rng(2)
+    W = bits(rng.standard_normal((N, K)))
+    X = correlated_calibration(3, M, K, rank=5)
+    u, s16, zp, W_pre = gptq.gptq_quantize(W, X, g, mode, return_trace=True)
+    What = gptq.dequantize(u, s16, zp, g)
+    w = f64(W)
+    x = f64(X)
+    XtX = x.T @ x
+    H = 2 * XtX + 0.01 * np.trace(XtX) / K * np.eye(K)
+    for j in range(1, K):
+        f, r = slice(0, j), slice(j, K)
+        e_f = w[:, f] - What[:, f]                         # [N, j]
+        # minimise (e_f, e_r) H (e_f, e_r)^T over e_r: H_rr e_r = -H_rf e_f
+        e_r = -np.linalg.solve(H[r, r], H[r, f] @ e_f.T)   # [K-j, N]
+        v = w[:, j] - e_r[0]
+        np.testing.assert_allclose(W_pre[:, j], v, rtol=1e-9, atol=1e-9 * np.abs(w).max())
+        if j % g == 0:
+            # the group's grid comes from all its columns as they stand now
+            # (the quantizer's pinned group rule applied to the solved state)
+            state = (w[:, j:j + g] - e_r[:g].T).astype(np.float32)
+            for n in range(N):
+                s, z, _ = oracle.quant_group(state[n], mode)
+                assert (s, z) == (int(s16[n, j // g]), int(zp[n, j // g])), (j, n)
+    np.testing.assert_array_equal(W_pre[:, 0], w[:, 0])
+
+
+def test_rank_one_hessian_closed_form():
+    # one calibration row x = (x0, x1): H = 2 x x^T + lam I with lam = 0.01 |x|^2 / 2.
+    # Quantizing column 0 with error e0 = w0 - w^0 moves column 1 by
+    #   -e0 [H^-1]_01 / [H^-1]_00 = e0 * 2 x0 x1 / (lam + 2 x1^2)   (Sherman-Morrison)
+    x0, x1 = 1.5, -0.75
+    X = bits([[x0, x1]])
+    W = bits([[0.3, -0.2], [0.11, 0.9], [-0.62, 0.05]])
+    u, s16, zp, W_pre = gptq.gptq_quantize(W, X, 2, ASYM, return_trace=True)
+    What = gptq.dequantize(u, s16, zp, 2)
+    w = f64(W)
+    lam = 0.01 * (x0 * x0 + x1 * x1) / 2
+    e0 = w[:, 0] - What[:, 0]
+    np.testing.assert_allclose(W_pre[:, 1], w[:, 1] + e0 * 2 * x0 * x1 / (lam + 2 * x1 * x1), rtol=1e-12)
+
+
+def test_no_calibration_signal_feeds_nothing_back():
+    W = bits(np.random.default_rng(4).standard_normal((3, 64)))
+    X = np.zeros((5, 64), dtype=np.uint16)
+    q, s, z = gptq.gptq_pack(W, X, 32, ASYM)
+    rq, rs, rz = oracle.quant_pack(W, 32, ASYM)
+    assert np.array_equal(q, rq) and np.array_equal(s, rs) and np.array_equal(z, rz)
+
+
+@pytest.mark.parametrize("mode", [SYM, ASYM])
+def test_grid_point_within_half_a_step(mode):
+    N, K, g = 6, 128, 32
+    W = bits(np.random.default_rng(5).standard_normal((N, K)))
+    X = correlated_calibration(6, 64, K, rank=8)
+    u, s16, zp, W_pre = gptq.gptq_quantize(W, X, g, mode, return_trace=True)
+    What = gptq.dequantize(u, s16, zp, g)
+    step = np.repeat(gptq.f16_bits_to_f64(s16), g, axis=1)
+    lo = np.repeat(0 - zp if mode == ASYM else np.full_like(zp, -8), g, axis=1) * step
+    hi = np.repeat(15 - zp if mode == ASYM else np.full_like(zp, 7), g, axis=1) * step
+    inside = (W_pre >= lo - step / 2) & (W_pre <= hi + step / 2)
+    slack = step * (0.5 + 2.0 ** -20) + 1e-30
+    assert np.all(np.abs(W_pre - What)[inside] <= slack[inside])
+    # outside the grid the code is the end point on that side
+    assert np.all(What[W_pre < lo - step / 2] == lo[W_pre < lo - step / 2])
+    assert np.all(What[W_pre > hi + step / 2] == hi[W_pre > hi + step / 2])
+
+
+def test_scene4_output_error_down_weight_error_up():
+    # INT4 g=64 on calibration features with low-rank correlation: the printed
+    # result is a 2.85x smaller output error with a larger weight error.
+    N, K, M, g = 64, 256, 512, 64
+    W = bits(np.random.default_rng(7).standard_normal((N, K)))
+    X = correlated_calibration(8, M, K, rank=16, noise=0.02)
+    u, s16, zp = gptq.gptq_quantize(W, X, g, ASYM)
+    What_g = gptq.dequantize(u, s16, zp, g)
+    q, s, z = oracle.quant_pack(W, g, ASYM)
+    What_r = oracle.dequant(q, s, z, K, g, ASYM, exact_f32=True).astype(np.float64)
+    w = f64(W)
+    werr = lambda Wh: np.linalg.norm(Wh - w) / np.linalg.norm(w)
+    out_g = gptq.output_error(W, What_g, X)
+    out_r = gptq.output_error(W, What_r, X)
+    assert out_g < out_r / 2
+    assert werr(What_g) > werr(What_r)
