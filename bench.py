@@ -562,10 +562,12 @@ def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps):
 
 # ------------------------------------------------------- oracle (CPU) ---
 
-def oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_per_weight: int, offset: int = 0):
+def oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_per_weight: int, offset: int = 0,
+                  threads: int = 1):
     """Run the oracle on rows [offset, offset + r) of each weight of the
     workload: quantize and pack, dequantize, and the fp64 product for those
-    output channels.  Returns the algorithmic bytes (or flops) processed."""
+    output channels (``threads`` row slices in parallel for the quantizer and
+    the product).  Returns the algorithmic bytes (or flops) processed."""
     nbytes = 0
     nflops = 0
     for k in keys:
@@ -573,13 +575,13 @@ def oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_per_weig
         W = host_W[k][0]
         r0 = offset % p.N
         r1 = min(p.N, r0 + rows_per_weight)
-        q, sc, z = oracle.quant_pack(W, p.group, p.mode, s=host_s[k], rows=(r0, r1))
+        q, sc, z = oracle.quant_pack(W, p.group, p.mode, s=host_s[k], rows=(r0, r1), threads=threads)
         nbytes += roofline.quant_pack_bytes(r1 - r0, p.K, p.group, p.mode, p.smooth)
         users = [pp for key, pp in plist if key == k and pp.M > 0]
         if users:
-            what = oracle.dequant(q, sc, z, p.K, p.group, p.mode, rows=(r0, r1))
+            what = oracle.dequant(q, sc, z, p.K, p.group, p.mode, rows=(r0, r1), threads=threads)
             for pp in users:
-                oracle.gemm_f64(host_X[pp.name][0], what)
+                oracle.gemm_f64(host_X[pp.name][0], what, threads=threads)
                 nbytes += roofline.gemm_bytes(pp.M, r1 - r0, pp.K, pp.group, pp.mode)
                 nflops += roofline.gemm_flops(pp.M, r1 - r0, pp.K)
     return nbytes, nflops
@@ -596,13 +598,23 @@ def cpu_baseline(workload, plist, keys, qp, host_W, host_X, host_s, budget_s):
     t0 = time.perf_counter()
     nbytes, nflops = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows)
     dt = time.perf_counter() - t0
-    if workload == "prefill":
-        val, unit = nflops / dt / 1e12, "TFLOP/s"
-    else:
-        val, unit = nbytes / dt / 1e9, "GB/s"
-    return {"value": val, "unit": unit, "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
-            "sample": "first %d rows of each weight of the workload: oracle fold+quantize+pack, dequantize and "
-                      "fp64 product for those output channels, single thread" % rows}
+    rate = lambda nb, nf, t: nf / t / 1e12 if workload == "prefill" else nb / t / 1e9
+    unit = "TFLOP/s" if workload == "prefill" else "GB/s"
+    out = {"value": rate(nbytes, nflops, dt), "unit": unit, "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
+           "sample": "first %d rows of each weight of the workload: oracle fold+quantize+pack, dequantize and "
+                     "fp64 product for those output channels, single thread" % rows}
+    cores = os.cpu_count() or 1
+    if cores > 1:
+        # the same oracle with its row slices spread over every host core
+        rows_mc = min(rows * cores, max(p.N for p in qp.values()))
+        t0 = time.perf_counter()
+        nb_mc, nf_mc = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_mc, threads=cores)
+        dt_mc = time.perf_counter() - t0
+        out["all_cores"] = {"value": rate(nb_mc, nf_mc, dt_mc), "unit": unit, "cores": cores,
+                            "seconds": round(dt_mc, 2),
+                            "sample": "first %d rows of each weight, the oracle's row slices on %d threads"
+                                      % (rows_mc, cores)}
+    return out
 
 
 def run_reference(args, rank, world):

@@ -160,7 +160,8 @@ def quant_pack(W_bits: np.ndarray, g: int, mode: int, s: np.ndarray | None = Non
 
 
 def dequant(qweight: np.ndarray, scales: np.ndarray, qzeros: np.ndarray | None, K: int, g: int,
-            mode: int, rows: tuple[int, int] | None = None, exact_f32: bool = False) -> np.ndarray:
+            mode: int, rows: tuple[int, int] | None = None, exact_f32: bool = False,
+            threads: int = 1) -> np.ndarray:
     """w^ = bf16_rne(float(u - zp) * float(s16)) (page 5 section 2.2, x^ = (q-zp)*s)
     for rows [r0, r1).  Returns bf16 bit patterns (uint16), or with
     ``exact_f32`` the exact fp32 product before the bf16 rounding."""
@@ -171,14 +172,21 @@ def dequant(qweight: np.ndarray, scales: np.ndarray, qzeros: np.ndarray | None, 
     if qzeros is not None:
         qzeros = np.ascontiguousarray(qzeros, dtype=np.uint32)
     L = lib()
-    if exact_f32:
-        out = np.zeros((r1 - r0, K), dtype=np.float32)
-        rc = L.orc_dequant_rows_f32(_ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, g, int(mode), r0, r1, _ptr(out))
+    out = np.zeros((r1 - r0, K), dtype=np.float32 if exact_f32 else np.uint16)
+    fn = L.orc_dequant_rows_f32 if exact_f32 else L.orc_dequant_rows
+
+    def run(span):
+        dst = out[span[0] - r0:span[1] - r0]       # rows of a C-contiguous array: contiguous
+        rc = fn(_ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, g, int(mode), span[0], span[1], _ptr(dst))
+        if rc != 0:
+            raise ValueError("oracle dequant rejected its arguments (code %d)" % rc)
+
+    spans = _chunks(r0, r1, threads)
+    if len(spans) == 1:
+        run(spans[0])
     else:
-        out = np.zeros((r1 - r0, K), dtype=np.uint16)
-        rc = L.orc_dequant_rows(_ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, g, int(mode), r0, r1, _ptr(out))
-    if rc != 0:
-        raise ValueError("oracle dequant rejected its arguments (code %d)" % rc)
+        with ThreadPoolExecutor(len(spans)) as ex:
+            list(ex.map(run, spans))
     return out
 
 

@@ -7,7 +7,7 @@ import pytest
 import torch.multiprocessing as mp
 
 import bench
-from bit_gemm_quant_b200 import roofline
+from bit_gemm_quant_b200 import roofline, synth
 
 
 def test_defaults_and_workloads():
@@ -87,3 +87,19 @@ def test_reference_arm_prints_one_complete_line(workload):
             bench.awq_desc(bench.AWQ_SHAPE["M"], bench.AWQ_SHAPE["N"], bench.AWQ_SHAPE["K"],
                            bench.AWQ_SHAPE["group"], bench.AWQ_SHAPE["n_alpha"]))
     assert d["config"]["workload"] == want
+
+
+def test_cpu_baseline_reports_single_thread_and_all_cores():
+    """The oracle timed single-threaded (the reported value) and, as a labelled
+    variant, with its row slices on every host core."""
+    plist = bench.problems_for("decode")
+    keys = list(dict.fromkeys(k for k, _ in plist))
+    qp = {k: p for k, p in reversed(plist)}
+    host_W = {k: [synth.weights(qp[k].seed, qp[k].N, qp[k].K, qp[k].w_std, *qp[k].w_outlier)] for k in keys}
+    host_s = {k: qp[k].s() for k in keys}
+    host_X = {p.name: [p.X()] for _, p in plist if p.M > 0}
+    cpu = bench.cpu_baseline("decode", plist, keys, qp, host_W, host_X, host_s, 0.3)
+    assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0 and cpu["unit"] == "GB/s"
+    if (os.cpu_count() or 1) > 1:
+        mc = cpu["all_cores"]
+        assert mc["cores"] == os.cpu_count() and mc["value"] > 0 and mc["unit"] == "GB/s"
