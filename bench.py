@@ -960,17 +960,7 @@ def run_fp4(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        oracle.build()
-        t0 = time.perf_counter()
-        oracle_fp4_sample(oracle, host_W, 16, 0)
-        dt = time.perf_counter() - t0
-        rows = min(N, max(16, int(16 * args.cpu_budget / max(dt, 1e-3))))
-        t0 = time.perf_counter()
-        nb = oracle_fp4_sample(oracle, host_W, rows, 0)
-        dt = time.perf_counter() - t0
-        cpu = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
-               "sample": "first %d rows of W[%d,%d], NVFP4 and MXFP4, oracle, single thread" % (rows, N, K)}
+        cpu = cpu_baseline_fp4(host_W, args.cpu_budget)
 
     if rank == 0:
         out = {
@@ -989,6 +979,23 @@ def run_fp4(args, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def cpu_baseline_fp4(host_W, budget_s):
+    """Both oracle quantizers on the first rows of the weight, single thread,
+    sized to about ``budget_s`` seconds."""
+    import oracle
+    oracle.build()
+    N, K = host_W.shape
+    t0 = time.perf_counter()
+    oracle_fp4_sample(oracle, host_W, 16, 0)
+    dt = time.perf_counter() - t0
+    rows = min(N, max(16, int(16 * budget_s / max(dt, 1e-3))))
+    t0 = time.perf_counter()
+    nb = oracle_fp4_sample(oracle, host_W, rows, 0)
+    dt = time.perf_counter() - t0
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
+            "sample": "first %d rows of W[%d,%d], NVFP4 and MXFP4, oracle, single thread" % (rows, N, K)}
 
 
 def fp4_e2e(w4, torch, device, host_W, steps):
