@@ -215,6 +215,9 @@ w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int64_t K, con
  *            low nibble of byte i, element 2i+1 in the high nibble.
  *   scales   out, uint8 [N][K/B]: E4M3 codes (NVFP4) or E8M0 codes (MXFP4).
  * Every output byte is written; outputs must not overlap inputs.
+ * Errors: W4_ERR_INVALID_ARG for a NULL or misaligned pointer, an unknown
+ * kind, N < 1, or K not a positive multiple of B; W4_ERR_CUDA if the launch
+ * fails.  Asynchronous on `stream`.
  */
 w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                        w4_stream_t stream);
