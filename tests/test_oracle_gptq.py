@@ -22,6 +22,7 @@ import numpy as np
 import pytest
 
 import oracle
+from conftest import golden
 from oracle import gptq
 from bit_gemm_quant_b200 import synth
 
@@ -137,6 +138,9 @@ def test_grid_point_within_half_a_step(mode):
 def test_scene4_output_error_down_weight_error_up():
     # INT4 g=64 on calibration features with low-rank correlation: the printed
     # result is a 2.85x smaller output error with a larger weight error.
+    fx = golden("gptq_scene4.json")["printed"]
+    assert fx["gptq"]["output_rel_l2"] < fx["rtn"]["output_rel_l2"] / 2
+    assert fx["gptq"]["weight_rel_l2"] > fx["rtn"]["weight_rel_l2"]
     N, K, M, g = 64, 256, 512, 64
     W = bits(np.random.default_rng(7).standard_normal((N, K)))
     X = correlated_calibration(8, M, K, rank=16, noise=0.02)
