@@ -3,23 +3,28 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl w4|reference] [--workload NAME]
 
-One step is one pass of the whole path over one batch of its workload: every
-weight matrix of the workload is quantized and packed (w4_quant_pack), and
-every activation batch is multiplied by its packed weight (w4a16_gemm).
+One step is one pass of the workload's kernels over one batch of its inputs.
+The product workloads (decode, smallbatch, prefill) multiply every activation
+batch by its packed weight (w4a16_gemm); their weights are quantized once,
+before the timed region, as a model's weights are at load time, and the
+GEMV-sized products are launched with W4_WEIGHTS_STATIC (the weight stream of
+one product may start before the previous kernel on the stream finishes).
+The quantizer workloads time the quantization itself.
 
   decode (default)  M=1, K=4096, N in {4096, 11008, 12288}, asymmetric INT4 g=128:
-                    3 x (w4_quant_pack + w4a16_gemm); value = algorithmic GB/s
-  smallbatch        K=8192, N=28672, symmetric g=128: 1 x w4_quant_pack + M in {2,4,8,16,32}
-  prefill           K=4096, N=14336, asymmetric g=128: 1 x w4_quant_pack + M in {512,2048,8192};
+                    3 x w4a16_gemm (GEMV); value = algorithmic GB/s
+  smallbatch        K=8192, N=28672, symmetric g=128: w4a16_gemm at M in {2,4,8,16,32}
+  prefill           K=4096, N=14336, asymmetric g=128: w4a16_gemm at M in {512,2048,8192};
                     value = GEMM TFLOP/s over the step
-  quantizer         W[28672, 8192]: g in {32,64,128} x {sym, asym} + smoothing fold
+  quantizer         w4_quant_pack of W[28672, 8192]: g in {32,64,128} x {sym, asym} + smoothing fold
+  decodequant       w4_quant_pack of the decode weights (K=4096, N in {4096, 11008, 12288}, asym g=128)
   awq               the AWQ scale search over W[4096, 4096] with 128 calibration rows
   fp4quant          W[28672, 8192] to NVFP4 and to MXFP4: 2 x w4_fp4_quant per step
 
 The K timed steps are captured in one CUDA graph (kernel nodes only) and
 replayed once between CUDA events on the launching stream.  Inputs rotate over
-two sets so that no kernel finds its inputs in the 126 MB L2: each GEMM reads
-the weights packed one step earlier, after more than 126 MB of other traffic.
+enough copies that no kernel finds its inputs in the 126 MB L2 (one sweep of
+the copies is more than 3x L2).
 Each kernel's device time is measured the same way, live: the median (and min)
 over five replays of a graph of max(K, 100) launches of that kernel alone over
 enough copies of its inputs (one sweep > 3x L2) that every launch reads them
@@ -65,7 +70,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["w4", "reference"], default="w4")
-    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "awq", "fp4quant"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "decodequant", "awq", "fp4quant"],
+                    default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -114,10 +120,15 @@ def problems_for(workload: str):
 
 
 WORKLOAD_DESC = {
-    "decode": "decode GEMV: M=1, K=4096, N in {4096,11008,12288}, asymmetric INT4 g=128, fp16 scales, uint4 zero-points; step = w4_quant_pack + w4a16_gemm per layer",
-    "smallbatch": "small-batch decode: K=8192, N=28672, symmetric INT4 g=128, M in {2,4,8,16,32}; step = 1 w4_quant_pack + 5 w4a16_gemm",
-    "prefill": "prefill GEMM: K=4096, N=14336, asymmetric INT4 g=128, M in {512,2048,8192}; step = 1 w4_quant_pack + 3 w4a16_gemm",
+    "decode": "decode GEMV: M=1, K=4096, N in {4096,11008,12288}, asymmetric INT4 g=128, fp16 scales, uint4 zero-points; "
+              "step = 3 w4a16_gemm (GEMV, W4_WEIGHTS_STATIC), weights quantized once before timing",
+    "smallbatch": "small-batch decode: K=8192, N=28672, symmetric INT4 g=128, M in {2,4,8,16,32}; "
+                  "step = 5 w4a16_gemm (W4_WEIGHTS_STATIC where M <= 16), weights quantized once before timing",
+    "prefill": "prefill GEMM: K=4096, N=14336, asymmetric INT4 g=128, M in {512,2048,8192}; step = 3 w4a16_gemm "
+               "(tensor cores), weights quantized once before timing",
     "quantizer": "quantizer sweep: W[28672,8192], g in {32,64,128} x {sym,asym} + smoothing fold; step = 7 w4_quant_pack",
+    "decodequant": "quantizer on the decode weights: W[N,4096] bf16, N in {4096,11008,12288}, asymmetric INT4 g=128; "
+                   "step = 3 w4_quant_pack",
     "fp4quant": "block-scaled FP4 weight quantization: W[28672,8192] bf16 to NVFP4 (E2M1, E4M3 scale per 16) and "
                 "to MXFP4 (E2M1, E8M0 scale per 32); step = 2 w4_fp4_quant",
 }
@@ -233,6 +244,9 @@ def traffic_table() -> dict:
 
 # ------------------------------------------------------------- our arm ---
 
+QUANT_WORKLOADS = ("quantizer", "decodequant")
+
+
 def run_w4(args, rank, world, local_rank):
     import torch
     import bit_gemm_quant_b200 as w4
@@ -245,60 +259,77 @@ def run_w4(args, rank, world, local_rank):
     w4.lib()
     pk = roofline.peaks(ROOT)
     plist = problems_for(args.workload)
-    R = 2  # rotating input sets
+    quant_step = args.workload in QUANT_WORKLOADS
     rank_seed = 1000 * rank
+    L2_BYTES = 126 << 20
 
     # ---- inputs (host bits, then device) ----
-    host_W, host_X, host_s = {}, {}, {}
-    for key, p in plist:
-        if key not in host_W:
-            host_W[key] = [synth.weights(p.seed + rank_seed + 17 * r, p.N, p.K, p.w_std, *p.w_outlier) for r in range(R)]
-            host_s[key] = p.s()
-        if p.M > 0:
-            host_X[p.name] = [synth.activations(p.seed + rank_seed + 17 * r, p.M, p.K, *p.x_outlier,
-                                                fixed_channels=p.x_fixed) for r in range(R)]
     keys = list(dict.fromkeys(k for k, _ in plist))
     first = {k: p for k, p in reversed(plist)}
-    qp = {k: first[k] for k in keys}     # the quantization problem of each weight key
+    qp = {k: first[k] for k in keys}              # the quantization problem of each weight key
+    host_W = {k: [synth.weights(qp[k].seed + rank_seed, qp[k].N, qp[k].K, qp[k].w_std, *qp[k].w_outlier)]
+              for k in keys}
+    host_s = {k: qp[k].s() for k in keys}
+    host_X = {p.name: [synth.activations(p.seed + rank_seed, p.M, p.K, *p.x_outlier, fixed_channels=p.x_fixed)]
+              for _, p in plist if p.M > 0}
 
     def dev_bf16(bits):
         return torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16)
 
-    W_d = {k: [dev_bf16(b) for b in host_W[k]] for k in keys}
+    W_d = {k: dev_bf16(host_W[k][0]) for k in keys}
     s_d = {k: (torch.from_numpy(host_s[k]).to(device) if host_s[k] is not None else None) for k in keys}
-    X_d = {n: [dev_bf16(b) for b in host_X[n]] for n in host_X}
-    packed = {}
-    for k in keys:
-        p = qp[k]
-        packed[k] = [w4.quant_pack(W_d[k][r], p.group, p.mode, s=s_d[k]) for r in range(R)]
-    Y_d, ws_d = {}, {}
-    for key, p in plist:
-        if p.M > 0:
-            Y_d[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device)
-            need = w4.w4a16_workspace_bytes(p.M, p.N, p.K, p.group)
-            ws_d[p.name] = torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
-    torch.cuda.synchronize()
+    X_d = {n: dev_bf16(v[0]) for n, v in host_X.items()}
+
+    def copies_for(nbytes):
+        return max(2, -(-3 * L2_BYTES // max(nbytes, 1)) + 1)   # reuse distance of one copy > 3x L2
+
+    def packed_bytes(p):
+        qs, ss, zs = w4.packed_shapes(p.N, p.K, p.group)
+        return qs[0] * qs[1] * 4 + ss[0] * ss[1] * 2 + (zs[0] * zs[1] * 4 if p.mode == w4.ASYM else 0)
 
     launches = []
-    for k in keys:
-        p = qp[k]
-        launches.append(Launch("w4_quant_pack", roofline.quant_pack_bytes(p.N, p.K, p.group, p.mode, p.smooth), 0,
-                               k))
-        for key, pp in plist:
-            if key == k and pp.M > 0:
-                launches.append(Launch(kernel_name(pp.M), roofline.gemm_bytes(pp.M, pp.N, pp.K, pp.group, pp.mode),
-                                       roofline.gemm_flops(pp.M, pp.N, pp.K), pp.name))
-
-    def step(si):
-        r, r_prev = si % R, (si + 1) % R
+    if quant_step:
+        # the quantizer reads each weight from one of several copies of W
+        W_pool = {k: [W_d[k]] + [W_d[k].clone() for _ in range(copies_for(W_d[k].numel() * 2) - 1)] for k in keys}
+        packed_out = {k: w4.quant_pack(W_d[k], qp[k].group, qp[k].mode, s=s_d[k]) for k in keys}
         for k in keys:
             p = qp[k]
-            w4.quant_pack(W_d[k][r], p.group, p.mode, s=s_d[k], out=packed[k][r])
-            for key, pp in plist:
-                if key == k and pp.M > 0:
-                    q, sc, z = packed[k][r_prev]
-                    w4.gemm(X_d[pp.name][r], q, sc, z, pp.group, pp.mode, N=pp.N, workspace=ws_d[pp.name],
-                            out=Y_d[pp.name])
+            launches.append(Launch("w4_quant_pack", roofline.quant_pack_bytes(p.N, p.K, p.group, p.mode, p.smooth), 0, k))
+    else:
+        # weights quantized once, as at model load; each product of a step takes
+        # the next of several copies of its packed weight
+        packed0 = {k: w4.quant_pack(W_d[k], qp[k].group, qp[k].mode, s=s_d[k]) for k in keys}
+        uses = {k: sum(1 for key, pp in plist if key == k and pp.M > 0) for k in keys}
+        P_pool = {}
+        for k in keys:
+            n = max(copies_for(packed_bytes(qp[k]) * uses[k]), uses[k] + 1)
+            P_pool[k] = [packed0[k]] + [tuple(None if t is None else t.clone() for t in packed0[k]) for _ in range(n - 1)]
+        Y_d, ws_d = {}, {}
+        for key, p in plist:
+            if p.M > 0:
+                Y_d[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device)
+                need = w4.w4a16_workspace_bytes(p.M, p.N, p.K, p.group)
+                ws_d[p.name] = torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
+                launches.append(Launch(kernel_name(p.M), roofline.gemm_bytes(p.M, p.N, p.K, p.group, p.mode),
+                                       roofline.gemm_flops(p.M, p.N, p.K), p.name))
+    torch.cuda.synchronize()
+
+    use_count = {k: 0 for k in keys}
+
+    def step(si):
+        if quant_step:
+            for k in keys:
+                p = qp[k]
+                pool = W_pool[k]
+                w4.quant_pack(pool[si % len(pool)], p.group, p.mode, s=s_d[k], out=packed_out[k])
+            return
+        for key, pp in plist:
+            if pp.M > 0:
+                pool = P_pool[key]
+                q, sc, z = pool[use_count[key] % len(pool)]
+                use_count[key] += 1
+                w4.gemm(X_d[pp.name], q, sc, z, pp.group, pp.mode, N=pp.N, workspace=ws_d[pp.name],
+                        out=Y_d[pp.name], weights_static=pp.M <= 16)
 
     per_step = len(launches)
     # ---- eager warm-up ----
@@ -354,10 +385,9 @@ def run_w4(args, rank, world, local_rank):
         clocks["remeasured"] = True
     del graph
 
-    # ---- per-kernel device time: each launch of the step alone, K times in one
-    # graph, over enough copies of its inputs (> 2x L2) that every launch reads
+    # ---- per-kernel device time: each launch of the step alone, KL times in one
+    # graph, over enough copies of its inputs (> 3x L2) that every launch reads
     # them from HBM; CUDA events on the launching stream around the replay ----
-    L2_BYTES = 126 << 20
     KL = max(K, 100)                             # launches per per-kernel graph
     REPLAYS = 5
 
@@ -386,28 +416,24 @@ def run_w4(args, rank, world, local_rank):
         del g
         return statistics.median(per), min(per)
 
-    def copies(ts, nbytes):
-        n = max(2, -(-3 * L2_BYTES // max(nbytes, 1)))   # one sweep > 3x L2
-        return [tuple(None if t is None else t.clone() for t in ts) for _ in range(n)]
-
     kt = {}
-    for k in keys:
-        p = qp[k]
-        W_pool = copies((W_d[k][0],), W_d[k][0].numel() * 2)
-        out = packed[k][0]
-        fns = [(lambda Wc=Wc: w4.quant_pack(Wc[0], p.group, p.mode, s=s_d[k], out=out)) for Wc in W_pool]
-        kt[("w4_quant_pack", k)] = kernel_graph_ms(fns)
-        del W_pool
-        for key, pp in plist:
-            if key == k and pp.M > 0:
-                q0, sc0, z0 = packed[k][0]
-                nb = q0.numel() * 4 + sc0.numel() * 2 + (0 if z0 is None else z0.numel() * 4)
-                P_pool = copies((q0, sc0, z0), nb)
-                fns = [(lambda Pc=Pc, pp=pp: w4.gemm(X_d[pp.name][0], Pc[0], Pc[1], Pc[2], pp.group, pp.mode,
-                                                     N=pp.N, workspace=ws_d[pp.name], out=Y_d[pp.name]))
-                       for Pc in P_pool]
-                kt[(kernel_name(pp.M), pp.name)] = kernel_graph_ms(fns)
-                del P_pool
+    for L in launches:
+        if quant_step:
+            p = qp[L.label]
+            fns = [(lambda Wc=Wc, p=p, k=L.label: w4.quant_pack(Wc, p.group, p.mode, s=s_d[k], out=packed_out[k]))
+                   for Wc in W_pool[L.label]]
+            kt[(L.name, L.label)] = kernel_graph_ms(fns)
+            continue
+        pp = next(p for _, p in plist if p.name == L.label)
+        key = next(k for k, p in plist if p.name == L.label)
+        pool = P_pool[key]
+        for static in ((True, False) if pp.M <= 16 else (False,)):
+            fns = [(lambda Pc=Pc, pp=pp, static=static: w4.gemm(X_d[pp.name], Pc[0], Pc[1], Pc[2], pp.group, pp.mode,
+                                                                 N=pp.N, workspace=ws_d[pp.name], out=Y_d[pp.name],
+                                                                 weights_static=static))
+                   for Pc in pool]
+            kt[(L.name, L.label, static)] = kernel_graph_ms(fns)
+        kt[(L.name, L.label)] = kt[(L.name, L.label, pp.M <= 16)]
     torch.cuda.synchronize()
 
     step_bytes = sum(L.bytes for L in launches)
@@ -431,9 +457,8 @@ def run_w4(args, rank, world, local_rank):
 
     kernels = {}
     by_name = {}
-    for L in launches:
-        avg, mn = kt[(L.name, L.label)]
-        ts = [avg] * KL
+
+    def entry(L, avg, mn):
         ent = {"launches": KL * REPLAYS, "avg_us": round(avg * 1e3, 3), "min_us": round(mn * 1e3, 3),
                "bytes": L.bytes,
                "gbs": round(L.bytes / (avg * 1e-3) / 1e9, 1),
@@ -443,8 +468,20 @@ def run_w4(args, rank, world, local_rank):
             peak_t = tensor_peak(avg)
             ent.update({"flops": L.flops, "tflops": round(tf, 1), "tensor_frac": round(tf / peak_t, 4),
                         "tensor_frac_burst": round(tf / pk["bf16_tflops"], 4)})
-        kernels["%s[%s]" % (L.name, L.label)] = ent
-        by_name.setdefault(L.name, []).append((L, ts))
+        return ent
+
+    for L in launches:
+        avg, mn = kt[(L.name, L.label)]
+        kernels["%s[%s]" % (L.name, L.label)] = entry(L, avg, mn)
+        if (L.name, L.label, False) in kt and (L.name, L.label, True) in kt:
+            # the same launch without W4_WEIGHTS_STATIC: the weight stream waits
+            # for the previous kernel to finish
+            kernels["%s[%s]" % (L.name, L.label)]["weights_static"] = True
+            a2, m2 = kt[(L.name, L.label, False)]
+            e2 = entry(L, a2, m2)
+            e2["weights_static"] = False
+            kernels["%s_plain[%s]" % (L.name, L.label)] = e2
+        by_name.setdefault(L.name, []).append((L, [avg] * KL))
 
     dom = max(by_name, key=lambda n: sum(sum(ts) for _, ts in by_name[n]))
     dom_launches = by_name[dom]
@@ -465,6 +502,10 @@ def run_w4(args, rank, world, local_rank):
         achieved = per_launch / (tot_time / nlaunch) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4)}
+    if dom == "w4a16_gemv":
+        roof["weights_static"] = True
+        plain = [kt[(L.name, L.label, False)][0] for L, _ in dom_launches]
+        roof["frac_plain"] = round(per_launch / (sum(plain) / len(plain) * 1e-3) / 1e9 / pk["hbm_gbs"], 4)
     tr = [traffic.get((dom, L.label)) for L, _ in dom_launches]
     roof["traffic"] = (sum(tr) / len(tr)) if tr and all(t is not None for t in tr) else None
     roof["kernel"] = dom
@@ -474,15 +515,15 @@ def run_w4(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, min(args.steps, 10))
+        e2e = run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, min(args.steps, 10), quant_step)
         e2e_ms, e2e_work = aggregate(e2e["ms"], e2e["work"] if args.workload != "prefill" else e2e["flops"], device)
         e2e = {"value": round(e2e_work / (e2e_ms * 1e-3) / (1e12 if args.workload == "prefill" else 1e9), 2),
                "unit": unit, "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-               "steps": e2e["steps"]}
+               "steps": e2e["steps"], "what": e2e["what"]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.workload, plist, keys, qp, host_W, host_X, host_s, args.cpu_budget)
+        cpu = cpu_baseline(args.workload, plist, keys, qp, host_W, host_X, host_s, args.cpu_budget, quant_step)
 
     if rank == 0:
         wl_desc = WORKLOAD_DESC[args.workload]
@@ -492,7 +533,7 @@ def run_w4(args, rank, world, local_rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": {"workload": wl_desc, "codes": "int4 packed 8 per uint32", "accumulate": "fp32",
-                       "l2": "inputs rotate over 2 sets; each kernel's inputs were last touched before >126 MB of other traffic",
+                       "l2": "every launch reads its weight from one of several copies whose reuse distance exceeds 3x L2",
                        "timing": "K steps captured in one CUDA graph (kernels only), replayed between CUDA events on the launching stream after %d untimed replays; max over ranks; per-kernel durations: median (and min) over 5 replays of a graph of max(K, 100) launches of that kernel alone over rotating input copies (one sweep > 3x L2), between CUDA events on its stream" % replays,
                        "parallelism": "replicas (dp%d), no data-path collective" % world},
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
@@ -504,46 +545,63 @@ def run_w4(args, rank, world, local_rank):
         dist.destroy_process_group()
 
 
-def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps):
-    """Same step through the tensor API with pinned host inputs and outputs:
-    host->device copies of each step's weights and activations, the library
-    calls, and device->host copies of the packed weights and Y, all timed."""
+def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps, quant_step):
+    """The step through the tensor API with pinned host buffers, all timed.
+    Quantizer workloads: host->device copies of W (and s), the quantization and
+    device->host copies of the packed weight.  Product workloads: the weights
+    are quantized once, untimed (model state); each step copies the
+    activations host->device, multiplies, and copies Y device->host."""
     pin = lambda a: torch.from_numpy(a.view(np.int16)).pin_memory()
-    hW = {k: pin(host_W[k][0]) for k in keys}
-    hX = {n: pin(v[0]) for n, v in host_X.items()}
-    hs = {k: (torch.from_numpy(host_s[k]).pin_memory() if host_s[k] is not None else None) for k in keys}
-    outs_q, outs_y = {}, {}
-    h2d = sum(hW[k].numel() * 2 + (hs[k].numel() * 4 if hs[k] is not None else 0) for k in keys) + \
-        sum(x.numel() * 2 for x in hX.values())
-    d2h = 0
-    for k in keys:
-        p = qp[k]
-        qs, ss, zs = w4.packed_shapes(p.N, p.K, p.group)
-        outs_q[k] = (torch.empty(qs, dtype=torch.int32).pin_memory(), torch.empty(ss, dtype=torch.float16).pin_memory(),
-                     torch.empty(zs, dtype=torch.int32).pin_memory() if p.mode == 1 else None)
-        d2h += sum(t.numel() * t.element_size() for t in outs_q[k] if t is not None)
-    for key, p in plist:
-        if p.M > 0:
-            outs_y[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
-            d2h += p.M * p.N * 2
-    work = sum(roofline.quant_pack_bytes(qp[k].N, qp[k].K, qp[k].group, qp[k].mode, qp[k].smooth) for k in keys) + \
-        sum(roofline.gemm_bytes(p.M, p.N, p.K, p.group, p.mode) for _, p in plist if p.M > 0)
-    flops = sum(roofline.gemm_flops(p.M, p.N, p.K) for _, p in plist if p.M > 0)
-
-    def one():
+    h2d = d2h = 0
+    if quant_step:
+        hW = {k: pin(host_W[k][0]) for k in keys}
+        hs = {k: (torch.from_numpy(host_s[k]).pin_memory() if host_s[k] is not None else None) for k in keys}
+        outs_q = {}
         for k in keys:
             p = qp[k]
-            Wd = hW[k].to(device, non_blocking=True).view(torch.bfloat16)
-            sd = hs[k].to(device, non_blocking=True) if hs[k] is not None else None
-            q, sc, z = w4.quant_pack(Wd, p.group, p.mode, s=sd)
-            for t_h, t_d in zip(outs_q[k], (q, sc, z)):
-                if t_h is not None:
-                    t_h.copy_(t_d, non_blocking=True)
+            qs, ss, zs = w4.packed_shapes(p.N, p.K, p.group)
+            outs_q[k] = (torch.empty(qs, dtype=torch.int32).pin_memory(),
+                         torch.empty(ss, dtype=torch.float16).pin_memory(),
+                         torch.empty(zs, dtype=torch.int32).pin_memory() if p.mode == 1 else None)
+            h2d += hW[k].numel() * 2 + (hs[k].numel() * 4 if hs[k] is not None else 0)
+            d2h += sum(t.numel() * t.element_size() for t in outs_q[k] if t is not None)
+        work = sum(roofline.quant_pack_bytes(qp[k].N, qp[k].K, qp[k].group, qp[k].mode, qp[k].smooth) for k in keys)
+        flops = 0
+
+        def one():
+            for k in keys:
+                p = qp[k]
+                Wd = hW[k].to(device, non_blocking=True).view(torch.bfloat16)
+                sd = hs[k].to(device, non_blocking=True) if hs[k] is not None else None
+                for t_h, t_d in zip(outs_q[k], w4.quant_pack(Wd, p.group, p.mode, s=sd)):
+                    if t_h is not None:
+                        t_h.copy_(t_d, non_blocking=True)
+        what = "H2D of W (and s), w4_quant_pack, D2H of the packed weight"
+    else:
+        packed = {}
+        for k in keys:
+            p = qp[k]
+            Wd = torch.from_numpy(host_W[k][0].view(np.int16)).to(device).view(torch.bfloat16)
+            sd = torch.from_numpy(host_s[k]).to(device) if host_s[k] is not None else None
+            packed[k] = w4.quant_pack(Wd, p.group, p.mode, s=sd)
+        hX = {n: pin(v[0]) for n, v in host_X.items()}
+        outs_y = {}
+        for key, p in plist:
+            if p.M > 0:
+                outs_y[p.name] = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
+                h2d += hX[p.name].numel() * 2
+                d2h += p.M * p.N * 2
+        work = sum(roofline.gemm_bytes(p.M, p.N, p.K, p.group, p.mode) for _, p in plist if p.M > 0)
+        flops = sum(roofline.gemm_flops(p.M, p.N, p.K) for _, p in plist if p.M > 0)
+
+        def one():
             for key, pp in plist:
-                if key == k and pp.M > 0:
+                if pp.M > 0:
+                    q, sc, z = packed[key]
                     Xd = hX[pp.name].to(device, non_blocking=True).view(torch.bfloat16)
                     Y = w4.gemm(Xd, q, sc, z, pp.group, pp.mode, N=pp.N)
                     outs_y[pp.name].copy_(Y, non_blocking=True)
+        what = "H2D of X, w4a16_gemm, D2H of Y (packed weights resident, quantized once before timing)"
 
     for _ in range(2):
         one()
@@ -557,59 +615,77 @@ def run_e2e(w4, torch, device, plist, keys, qp, host_W, host_X, host_s, steps):
     e1.synchronize()
     barrier()
     ms = e0.elapsed_time(e1)
-    return {"ms": ms, "work": work * steps, "flops": flops * steps, "h2d": h2d, "d2h": d2h, "steps": steps}
+    return {"ms": ms, "work": work * steps, "flops": flops * steps, "h2d": h2d, "d2h": d2h, "steps": steps,
+            "what": what}
 
 
 # ------------------------------------------------------- oracle (CPU) ---
 
+def oracle_prepare(oracle, keys, qp, host_W, host_s, rows_per_weight: int, offset: int = 0, threads: int = 1):
+    """Quantize rows [offset, offset + r) of each weight with the oracle and
+    dequantize them (the product workloads' model state, not timed)."""
+    out = {}
+    for k in keys:
+        p = qp[k]
+        r0 = offset % p.N
+        r1 = min(p.N, r0 + rows_per_weight)
+        q, sc, z = oracle.quant_pack(host_W[k][0], p.group, p.mode, s=host_s[k], rows=(r0, r1), threads=threads)
+        out[k] = oracle.dequant(q, sc, z, p.K, p.group, p.mode, rows=(r0, r1), threads=threads), r1 - r0
+    return out
+
+
 def oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_per_weight: int, offset: int = 0,
-                  threads: int = 1):
-    """Run the oracle on rows [offset, offset + r) of each weight of the
-    workload: quantize and pack, dequantize, and the fp64 product for those
-    output channels (``threads`` row slices in parallel for the quantizer and
-    the product).  Returns the algorithmic bytes (or flops) processed."""
+                  threads: int = 1, quant_step: bool = False, prepared=None):
+    """The oracle's share of one step on rows [offset, offset + r) of each
+    weight: quantize and pack them (quantizer workloads), or the fp64 product
+    of the activations with those output channels of the dequantized weight
+    (product workloads; ``prepared`` from oracle_prepare).  Returns the
+    algorithmic bytes (or flops) processed."""
     nbytes = 0
     nflops = 0
     for k in keys:
         p = qp[k]
-        W = host_W[k][0]
-        r0 = offset % p.N
-        r1 = min(p.N, r0 + rows_per_weight)
-        q, sc, z = oracle.quant_pack(W, p.group, p.mode, s=host_s[k], rows=(r0, r1), threads=threads)
-        nbytes += roofline.quant_pack_bytes(r1 - r0, p.K, p.group, p.mode, p.smooth)
-        users = [pp for key, pp in plist if key == k and pp.M > 0]
-        if users:
-            what = oracle.dequant(q, sc, z, p.K, p.group, p.mode, rows=(r0, r1), threads=threads)
-            for pp in users:
-                oracle.gemm_f64(host_X[pp.name][0], what, threads=threads)
-                nbytes += roofline.gemm_bytes(pp.M, r1 - r0, pp.K, pp.group, pp.mode)
-                nflops += roofline.gemm_flops(pp.M, r1 - r0, pp.K)
+        if quant_step:
+            r0 = offset % p.N
+            r1 = min(p.N, r0 + rows_per_weight)
+            oracle.quant_pack(host_W[k][0], p.group, p.mode, s=host_s[k], rows=(r0, r1), threads=threads)
+            nbytes += roofline.quant_pack_bytes(r1 - r0, p.K, p.group, p.mode, p.smooth)
+            continue
+        what, nr = prepared[k]
+        for pp in (pp for key, pp in plist if key == k and pp.M > 0):
+            oracle.gemm_f64(host_X[pp.name][0], what, threads=threads)
+            nbytes += roofline.gemm_bytes(pp.M, nr, pp.K, pp.group, pp.mode)
+            nflops += roofline.gemm_flops(pp.M, nr, pp.K)
     return nbytes, nflops
 
 
-def cpu_baseline(workload, plist, keys, qp, host_W, host_X, host_s, budget_s):
+def cpu_baseline(workload, plist, keys, qp, host_W, host_X, host_s, budget_s, quant_step):
     import oracle
     oracle.build()
-    t0 = time.perf_counter()
-    oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, 4)
-    dt = time.perf_counter() - t0
-    rows = max(4, int(4 * budget_s / max(dt, 1e-3)))
-    rows = min(rows, max(p.N for p in qp.values()))
-    t0 = time.perf_counter()
-    nbytes, nflops = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows)
-    dt = time.perf_counter() - t0
     rate = lambda nb, nf, t: nf / t / 1e12 if workload == "prefill" else nb / t / 1e9
     unit = "TFLOP/s" if workload == "prefill" else "GB/s"
+    maxrows = max(p.N for p in qp.values())
+
+    def timed(rows, threads):
+        prep = None if quant_step else oracle_prepare(oracle, keys, qp, host_W, host_s, rows, threads=threads)
+        t0 = time.perf_counter()
+        nb, nf = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, threads=threads,
+                               quant_step=quant_step, prepared=prep)
+        return nb, nf, time.perf_counter() - t0
+
+    _, _, dt = timed(4, 1)
+    rows = min(maxrows, max(4, int(4 * budget_s / max(dt, 1e-3))))
+    nbytes, nflops, dt = timed(rows, 1)
+    what = ("oracle fold+quantize+pack" if quant_step else
+            "oracle fp64 product of the activations with those output channels of the dequantized weight "
+            "(quantized by the oracle beforehand, untimed)")
     out = {"value": rate(nbytes, nflops, dt), "unit": unit, "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
-           "sample": "first %d rows of each weight of the workload: oracle fold+quantize+pack, dequantize and "
-                     "fp64 product for those output channels, single thread" % rows}
+           "sample": "first %d rows of each weight of the workload: %s, single thread" % (rows, what)}
     cores = os.cpu_count() or 1
     if cores > 1:
         # the same oracle with its row slices spread over every host core
-        rows_mc = min(rows * cores, max(p.N for p in qp.values()))
-        t0 = time.perf_counter()
-        nb_mc, nf_mc = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows_mc, threads=cores)
-        dt_mc = time.perf_counter() - t0
+        rows_mc = min(rows * cores, maxrows)
+        nb_mc, nf_mc, dt_mc = timed(rows_mc, cores)
         out["all_cores"] = {"value": rate(nb_mc, nf_mc, dt_mc), "unit": unit, "cores": cores,
                             "seconds": round(dt_mc, 2),
                             "sample": "first %d rows of each weight, the oracle's row slices on %d threads"
@@ -630,24 +706,35 @@ def run_reference(args, rank, world):
     keys = list(dict.fromkeys(k for k, _ in plist))
     first = {k: p for k, p in reversed(plist)}
     qp = {k: first[k] for k in keys}
+    quant_step = args.workload in QUANT_WORKLOADS
     host_W = {k: [synth.weights(qp[k].seed, qp[k].N, qp[k].K, qp[k].w_std, *qp[k].w_outlier)] for k in keys}
     host_s = {k: qp[k].s() for k in keys}
     host_X = {p.name: [p.X()] for _, p in plist if p.M > 0}
     rows = 8
+    steps_total = max(3, args.warmup) + args.steps
+    # the product workloads' model state: every sampled row quantized and
+    # dequantized by the oracle before timing
+    prep = {} if quant_step else {
+        si: oracle_prepare(oracle, keys, qp, host_W, host_s, rows, si * rows) for si in range(steps_total)}
     for si in range(max(3, args.warmup)):
-        oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, si * rows)
+        oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, si * rows, quant_step=quant_step,
+                      prepared=prep.get(si))
     nb = nf = 0
     t0 = time.perf_counter()
-    for si in range(args.steps):
-        b, f = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, si * rows)
+    for j in range(args.steps):
+        si = max(3, args.warmup) + j
+        b, f = oracle_sample(oracle, plist, keys, qp, host_W, host_X, host_s, rows, si * rows, quant_step=quant_step,
+                             prepared=prep.get(si))
         nb, nf = nb + b, nf + f
     dt = time.perf_counter() - t0
     if args.workload == "prefill":
         val, unit = nf / dt / 1e12, "TFLOP/s"
     else:
         val, unit = nb / dt / 1e9, "GB/s"
-    sample = ("%d rows of each weight per step (rotating): oracle fold+quantize+pack, dequantize and fp64 "
-              "product for those output channels, single thread" % rows)
+    what = ("oracle fold+quantize+pack" if quant_step else
+            "oracle fp64 product with those output channels of the dequantized weight (quantized by the oracle "
+            "before timing)")
+    sample = "%d rows of each weight per step (rotating): %s, single thread" % (rows, what)
     print_reference(args, world, val, unit, dt * 1e3 / args.steps, WORKLOAD_DESC[args.workload], sample)
 
 

@@ -14,6 +14,9 @@ import ctypes
 import os
 
 SYM, ASYM = 0, 1
+# OR-ed into the mode of w4a16_gemm / w4a16_gemm_noalloc: the packed weight is
+# not written by the kernel right before the call on the stream (include/w4.h)
+WEIGHTS_STATIC = 0x100
 NVFP4, MXFP4 = 0, 1
 FP4_BLOCK = {NVFP4: 16, MXFP4: 32}
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
@@ -145,8 +148,12 @@ def quant_pack(W, group: int = 128, mode: int = SYM, s=None, stream=None, out=No
 
 
 def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None, workspace=None,
-         out=None, stream=None):
-    """Y[M,N] = X . W^T from the packed weight; X bf16 CUDA tensor [M,K]."""
+         out=None, stream=None, weights_static: bool = False):
+    """Y[M,N] = X . W^T from the packed weight; X bf16 CUDA tensor [M,K].
+    ``weights_static`` passes W4_WEIGHTS_STATIC: the caller declares that the
+    kernel right before this call on the stream does not write the packed
+    weight (weights quantized once, earlier), so the weight stream may start
+    before that kernel finishes."""
     import torch
     M, K = X.shape
     if N is None:
@@ -156,8 +163,9 @@ def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None
     if need and workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=X.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = w4a16_gemm(_ptr(X), M, N, K, _ptr(qweight), _ptr(scales), _ptr(qzeros), group, mode, _ptr(Y),
-                    _ptr(workspace), wbytes, _stream_handle(stream))
+    st = w4a16_gemm(_ptr(X), M, N, K, _ptr(qweight), _ptr(scales), _ptr(qzeros), group,
+                    mode | (WEIGHTS_STATIC if weights_static else 0), _ptr(Y), _ptr(workspace), wbytes,
+                    _stream_handle(stream))
     if st != W4_OK:
         raise W4Error(st, "w4a16_gemm")
     return Y

@@ -11,13 +11,22 @@ bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
 
 bool mode_ok(int m) { return m == W4_SYM || m == W4_ASYM; }
 
-// batches up to this size run the GEMV (two MMA token groups of 8)
-constexpr int64_t kGemvMaxM = 16;
-
 // int64 products used for sizes must not overflow
 bool fits(int64_t a, int64_t b) { return a > 0 && b > 0 && a <= INT64_MAX / b; }
 
 }  // namespace
+
+namespace w4 {
+
+bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= kGemvMaxM) return N <= INT32_MAX - 16 && K <= INT32_MAX && M * K <= INT32_MAX;
+    // tensor-core path: 32-bit indices, TMA extents
+    return M <= INT32_MAX && N <= INT32_MAX && K <= INT32_MAX && M * K <= INT32_MAX &&
+           (int64_t)N * K / 8 <= INT32_MAX * 4LL;
+}
+
+}  // namespace w4
 
 extern "C" {
 
@@ -65,7 +74,7 @@ w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *c
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group)
 {
     (void)group;
-    if (M <= kGemvMaxM || M < 1 || N < 1 || K < 1) return 0;
+    if (M <= w4::kGemvMaxM || M < 1 || N < 1 || K < 1) return 0;
     return w4::tc_workspace_bytes(M, N, K);
 }
 
@@ -73,6 +82,8 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
                      const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
                      void *workspace, size_t workspace_bytes, w4_stream_t stream)
 {
+    const bool weights_static = (mode & W4_WEIGHTS_STATIC) != 0;
+    mode &= ~W4_WEIGHTS_STATIC;
     if (!X || !qweight || !scales || !Y) return W4_ERR_INVALID_ARG;
     if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N))
@@ -84,16 +95,13 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
     const size_t need = w4a16_workspace_bytes(M, N, K, group);
     if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256))))
         return W4_ERR_INVALID_ARG;
+    if (!w4::gemm_shape_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
     cudaError_t e;
-    if (M <= kGemvMaxM) {
-        if (N > INT32_MAX - 16 || K > INT32_MAX || M * K > INT32_MAX) return W4_ERR_UNSUPPORTED;
-        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, Y, (cudaStream_t)stream);
-    } else {
-        // tensor-core path: 32-bit indices, TMA extents
-        if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX || M * K > INT32_MAX || (int64_t)N * K / 8 > INT32_MAX * 4LL)
-            return W4_ERR_UNSUPPORTED;
+    if (M <= w4::kGemvMaxM)
+        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, weights_static, Y,
+                            (cudaStream_t)stream);
+    else
         e = w4::launch_gemm_tc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace, (cudaStream_t)stream);
-    }
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 

@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "w4.h"
@@ -64,8 +65,29 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_fl
 cudaError_t launch_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode, const float *s,
                               uint32_t *qweight, void *scales, uint32_t *qzeros, cudaStream_t stream);
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
-                        const void *scales, const uint32_t *qzeros, int group, int mode, void *Y,
+                        const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static, void *Y,
                         cudaStream_t stream);
+// Batches up to this size run the GEMV (two MMA token groups of 8); larger ones
+// the tensor-core kernel.
+constexpr int64_t kGemvMaxM = 16;
+// Shapes the product's kernels cannot index (32-bit indices, TMA extents).
+bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
+// Opt a kernel into `bytes` of dynamic shared memory on the current device.
+// The attribute is per device, so the flag that skips repeated calls is kept
+// per device too (an array indexed by the device ordinal).
+constexpr int kMaxDevices = 64;
+template <typename Kern>
+cudaError_t set_smem_attr(Kern kern, int bytes, std::atomic<bool> (&done)[kMaxDevices])
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+    return e;
+}
 cudaError_t launch_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                              cudaStream_t stream);
 size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);

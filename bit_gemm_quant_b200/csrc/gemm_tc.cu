@@ -509,12 +509,10 @@ cudaError_t launch_bn(const CUtensorMap &map, const CUtensorMap &qmap, const CUt
     using C = TcCfg<BN>;
     size_t smem = 1024 + C::kStages * C::kStageBytes + 256;
     if (C::kMinBlocks == 2 && smem < 80 * 1024) smem = 80 * 1024;   // at most 2 CTAs share an SM's tensor memory
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)smem);
+    static std::atomic<bool> attr_done[kMaxDevices];   // the attribute is per device
+    {
+        const cudaError_t e = set_smem_attr(gemm_tc_kernel<BN>, (int)smem, attr_done);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     float *partial = nullptr;
     unsigned *counters = nullptr;

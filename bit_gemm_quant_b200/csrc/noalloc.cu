@@ -29,8 +29,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[W4_NOALLOC_SCRA
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::atomic<void *> g_scratch_addr[kMaxDevices];
+std::atomic<void *> g_scratch_addr[w4::kMaxDevices];
 
 // Device address of the scratch array on the current device, resolved on the
 // first call for that device.
@@ -39,7 +38,7 @@ cudaError_t scratch_address(void **out)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= w4::kMaxDevices) return cudaErrorInvalidDevice;
     void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
     if (!p) {
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
@@ -59,6 +58,7 @@ bool fits(int64_t a, int64_t b) { return a > 0 && b > 0 && a <= INT64_MAX / b; }
 bool args_ok(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight, const void *scales,
              const uint32_t *qzeros, int group, int mode, const void *Y)
 {
+    mode &= ~W4_WEIGHTS_STATIC;
     if (!X || !qweight || !scales || !Y) return false;
     if (!(group == 32 || group == 64 || group == 128) || !(mode == W4_SYM || mode == W4_ASYM)) return false;
     if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N)) return false;
@@ -75,6 +75,8 @@ extern "C" w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int
                                         w4_stream_t stream)
 {
     if (!args_ok(X, M, N, K, qweight, scales, qzeros, group, mode, Y)) return W4_ERR_INVALID_ARG;
+    // every rejection happens before anything is enqueued, the counter clear included
+    if (!w4::gemm_shape_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
     const size_t need = w4a16_workspace_bytes(M, N, K, group);
     if (need > (size_t)W4_NOALLOC_SCRATCH_BYTES) return W4_ERR_UNSUPPORTED;
     void *scratch = nullptr;

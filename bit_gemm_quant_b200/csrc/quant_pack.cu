@@ -578,13 +578,11 @@ cudaError_t launch_variant(const CUtensorMap &map, const void *W, int64_t N, int
                            cudaStream_t stream)
 {
     const int threads = 256;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(quant_pack_kernel<G, MODE, FOLD, TMA>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   2048 + kQRingBytes + kMaxStagedS);
+    static std::atomic<bool> attr_done[kMaxDevices];   // the attribute is per device
+    {
+        const cudaError_t e =
+            set_smem_attr(quant_pack_kernel<G, MODE, FOLD, TMA>, 2048 + kQRingBytes + kMaxStagedS, attr_done);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     int per_sm = 0;                              // resident blocks per SM at this shared-memory size
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_pack_kernel<G, MODE, FOLD, TMA>, threads, smem) !=

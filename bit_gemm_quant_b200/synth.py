@@ -23,6 +23,7 @@ SmoothQuant sections of the pages):
   quantizer   W[28672,8192] ~ N(0,0.02); g in {32,64,128} x {sym, asym}; plus
               the smoothing fold with s = act^0.5/mean(act^0.5),
               act = |N(0,1)| with 1% of channels x20.
+  decodequant the decode workload's three weights, quantized (no product).
 
 "p% outlier channels" are the first round(p*K) entries of a seeded
 permutation of 0..K-1; weight columns and activation channels are drawn
@@ -140,6 +141,10 @@ def workload(name: str) -> list[Problem]:
     if name == "prefill":
         return [Problem("prefill_M%d" % M, M, 14336, 4096, 128, ASYM, 0.02, (0.0, 1.0), (0.01, 40.0), seed=3)
                 for M in (512, 2048, 8192)]
+    if name == "decodequant":
+        # the decode layers' weights (same seeds as the decode workload), quantized
+        return [Problem("decode_N%d" % N, 0, N, 4096, 128, ASYM, 0.02, (0.01, 5.0), seed=1)
+                for N in (4096, 11008, 12288)]
     if name == "quantizer":
         probs = []
         for g in (32, 64, 128):
@@ -151,4 +156,4 @@ def workload(name: str) -> list[Problem]:
     raise KeyError(name)
 
 
-WORKLOADS = ("tiny", "decode", "smallbatch", "prefill", "quantizer")
+WORKLOADS = ("tiny", "decode", "smallbatch", "prefill", "quantizer", "decodequant")

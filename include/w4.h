@@ -78,6 +78,21 @@ typedef enum {
 
 typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
 
+/*
+ * W4_WEIGHTS_STATIC -- a flag OR-ed into the `mode` argument of w4a16_gemm and
+ * w4a16_gemm_noalloc (never of w4_quant_pack).  It declares that the packed
+ * weight, its scales and its zero-points are NOT written by the kernel that
+ * immediately precedes this call on `stream` -- the usual case for model
+ * weights quantized once at load time.  The product may then start reading
+ * the weight before that kernel has finished (programmatic dependent launch;
+ * only the activations wait for it), so in a decode loop the weight stream of
+ * one layer overlaps the tail of the previous kernel.  The results are the
+ * same bits as without the flag.  If the declaration is false (the weight is
+ * quantized by the kernel right before this call, on the same stream), the
+ * result is undefined.  The tensor-core path (M > 16) ignores the flag.
+ */
+#define W4_WEIGHTS_STATIC 0x100
+
 /* Block-scaled FP4 kinds for w4_fp4_quant. */
 typedef enum { W4_NVFP4 = 0, W4_MXFP4 = 1 } w4_fp4_kind;
 
@@ -121,6 +136,7 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
  *   workspace, workspace_bytes: device scratch of at least
  *            w4a16_workspace_bytes(M, N, K, group) bytes (may be NULL when
  *            that is 0); 256-byte aligned.
+ *   mode     W4_SYM or W4_ASYM, optionally OR-ed with W4_WEIGHTS_STATIC.
  * Paths: M <= 16 runs the GEMV (codes streamed to shared memory by TMA,
  * dequantized in registers, mma.sync); larger M runs the tcgen05 kernel
  * (dequantized weights in tensor memory, activations in shared memory, fp32

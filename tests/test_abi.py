@@ -171,3 +171,29 @@ def test_awq_search_rejects_malformed_arguments_before_any_launch(w4):
     assert call(wsb=1024) == E                   # workspace too small
     assert call(K=500) == E
     assert call(s=P + 4) == E
+
+
+def test_weights_static_flag_is_accepted_only_in_the_product_mode(w4):
+    """W4_WEIGHTS_STATIC is stripped from the product's mode before the mode is
+    checked (a well-formed flagged call fails only for its other defects); any
+    other bit, or the flag on the quantizer, is an invalid mode."""
+    E = w4.W4_ERR_INVALID_ARG
+    flag = w4.WEIGHTS_STATIC
+    m = re.search(r"#define\s+W4_WEIGHTS_STATIC\s+(0x[0-9a-fA-F]+)", open(HEADER).read())
+    assert int(m.group(1), 16) == flag
+    assert mm(w4, mode=w4.ASYM | flag) == E                  # asymmetric without qzeros: the mode was read as ASYM
+    assert mm(w4, mode=w4.SYM | flag, z=FAKE) == E           # symmetric with qzeros: read as SYM
+    assert mm(w4, mode=0x200) == E                           # an unknown bit
+    assert mm(w4, mode=flag | 0x200) == E
+    assert qp(w4, mode=flag) == E                            # the quantizer has no such flag
+
+
+def test_noalloc_rejects_an_unsupported_shape_before_enqueuing_anything(w4):
+    """A shape outside the kernels' index range is rejected on the host, before
+    the entry point enqueues its counter clear (fake pointers: nothing may touch
+    them, and no CUDA call may be made on a machine without a GPU)."""
+    U = w4.W4_ERR_UNSUPPORTED
+    st = w4.w4a16_gemm_noalloc(P(FAKE), 64, 128, 1 << 26, P(FAKE), P(FAKE), None, 128, 0, P(FAKE), None)
+    assert st == U
+    need = w4.w4a16_workspace_bytes(64, 128, 1 << 26, 128)
+    assert mm(w4, M=64, N=128, K=1 << 26, ws=FAKE, wsb=need) == U   # w4a16_gemm agrees

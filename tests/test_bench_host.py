@@ -62,7 +62,7 @@ def test_max_over_ranks_gloo():
         assert ms == 15.0 and units == 300.0
 
 
-@pytest.mark.parametrize("workload", ["decode", "awq", "fp4quant"])
+@pytest.mark.parametrize("workload", ["decode", "decodequant", "awq", "fp4quant"])
 def test_reference_arm_prints_one_complete_line(workload):
     """`bench.py --impl reference` (the CPU oracle on a bounded sample) prints
     one JSON line with the base contract's keys and the same workload
@@ -89,17 +89,22 @@ def test_reference_arm_prints_one_complete_line(workload):
     assert d["config"]["workload"] == want
 
 
-def test_cpu_baseline_reports_single_thread_and_all_cores():
+@pytest.mark.parametrize("workload", ["decode", "decodequant"])
+def test_cpu_baseline_reports_single_thread_and_all_cores(workload):
     """The oracle timed single-threaded (the reported value) and, as a labelled
-    variant, with its row slices on every host core."""
-    plist = bench.problems_for("decode")
+    variant, with its row slices on every host core: the product for the
+    product workloads (weights quantized by the oracle beforehand), the
+    quantization for the quantizer workloads."""
+    plist = bench.problems_for(workload)
     keys = list(dict.fromkeys(k for k, _ in plist))
     qp = {k: p for k, p in reversed(plist)}
     host_W = {k: [synth.weights(qp[k].seed, qp[k].N, qp[k].K, qp[k].w_std, *qp[k].w_outlier)] for k in keys}
     host_s = {k: qp[k].s() for k in keys}
     host_X = {p.name: [p.X()] for _, p in plist if p.M > 0}
-    cpu = bench.cpu_baseline("decode", plist, keys, qp, host_W, host_X, host_s, 0.3)
+    quant = workload in bench.QUANT_WORKLOADS
+    cpu = bench.cpu_baseline(workload, plist, keys, qp, host_W, host_X, host_s, 0.3, quant)
     assert cpu["kind"] == "oracle" and cpu["cores"] == 1 and cpu["value"] > 0 and cpu["unit"] == "GB/s"
+    assert ("fold+quantize+pack" in cpu["sample"]) == quant
     if (os.cpu_count() or 1) > 1:
         mc = cpu["all_cores"]
         assert mc["cores"] == os.cpu_count() and mc["value"] > 0 and mc["unit"] == "GB/s"

@@ -183,3 +183,30 @@ def test_smallbatch_workload_sampled(w4, prob):
     Y = gpu_path(w4, W, X, prob.group, prob.mode)
     ch = np.sort(np.random.default_rng(77).choice(prob.N, 1024, replace=False))
     assert_y_close(Y[:, ch], oracle_ref(W, X, prob.group, prob.mode, channels=ch))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K,g,mode", [(1, 4096, 4096, 128, ASYM), (1, 12288, 4096, 128, ASYM),
+                                           (1, 11008, 4096, 128, ASYM), (4, 200, 1152, 128, SYM),
+                                           (8, 28672, 8192, 128, SYM), (13, 1000, 2304, 64, ASYM),
+                                           (2, 37904, 256, 32, SYM)])
+def test_weights_static_flag_gives_the_same_bits(w4, M, N, K, g, mode):
+    """W4_WEIGHTS_STATIC only lets the weight stream start before the previous
+    kernel on the stream finishes: with the weight quantized (and synchronized)
+    beforehand, the flagged product gives exactly the unflagged bits, on every
+    launch shape of the GEMV (few tiles, five and six tiles per SM, two token
+    groups, one-box rows), in a chain of back-to-back products."""
+    import torch
+    W = synth.weights(M + N + K, N, K, 0.02, 0.01, 5.0)
+    X = synth.activations(M + N + K, M, K, 0.01, 40.0)
+    q, sc, z = w4.quant_pack(dev_bf16(W), g, mode)
+    Xd = dev_bf16(X)
+    torch.cuda.synchronize()
+    ref = host_bf16_as_f64(w4.gemm(Xd, q, sc, z, g, mode))
+    outs = [w4.gemm(Xd, q, sc, z, g, mode, weights_static=True) for _ in range(4)]
+    torch.cuda.synchronize()
+    for Y in outs:
+        assert np.array_equal(host_bf16_as_f64(Y), ref)
+    assert w4.w4_device_error() == 0
+    if M * N <= 300000:
+        check(ref, W, X, g, mode)
