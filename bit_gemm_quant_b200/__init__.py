@@ -59,6 +59,10 @@ def lib() -> ctypes.CDLL:
         L.w4_layout_version.restype = I
         L.w4_device_error.argtypes = [ctypes.POINTER(I)]
         L.w4_device_error.restype = I
+        L.w4_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.w4_set_wait_limit_ns.restype = None
+        L.w4_test_stall_first_wait.argtypes = [I]
+        L.w4_test_stall_first_wait.restype = None
         _lib = L
     return _lib
 
@@ -102,6 +106,14 @@ def w4_status_string(status: int) -> str:
 
 def w4_layout_version() -> int:
     return int(lib().w4_layout_version())
+
+
+def w4_set_wait_limit_ns(ns: int) -> None:
+    lib().w4_set_wait_limit_ns(int(ns))
+
+
+def w4_test_stall_first_wait(on: int) -> None:
+    lib().w4_test_stall_first_wait(int(on))
 
 
 def w4_device_error() -> int:

@@ -18,6 +18,17 @@ bool fits(int64_t a, int64_t b) { return a > 0 && b > 0 && a <= INT64_MAX / b; }
 
 namespace w4 {
 
+namespace {
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitNs};
+std::atomic<int> g_stall_first_wait{0};
+}
+
+uint64_t wait_limit_ns()
+{
+    return g_wait_limit_ns.load(std::memory_order_relaxed) |
+           (g_stall_first_wait.load(std::memory_order_relaxed) ? kStallFirstWait : 0);
+}
+
 bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
 {
     if (M <= kGemvMaxM) return N <= INT32_MAX - 16 && K <= INT32_MAX && M * K <= INT32_MAX;
@@ -131,6 +142,14 @@ w4_status w4_awq_search(const void *W, const void *X, int64_t N, int64_t K, int6
                                                 workspace, (cudaStream_t)stream);
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
+
+void w4_set_wait_limit_ns(uint64_t ns)
+{
+    ns = ns == 0 ? w4::kDefaultWaitNs : ns;
+    w4::g_wait_limit_ns.store(ns > w4::kDefaultWaitNs ? w4::kDefaultWaitNs : ns, std::memory_order_relaxed);
+}
+
+void w4_test_stall_first_wait(int on) { w4::g_stall_first_wait.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 w4_status w4_device_error(int *code)
 {

@@ -100,6 +100,18 @@ size_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode,
 cudaError_t launch_awq_search(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
                               int n_alpha, double *losses, int *best, float *s_best, void *ws, cudaStream_t stream);
 int read_and_clear_device_error();
+// Time after which a kernel's wait for a copy, an MMA or another warp gives up
+// (default kDefaultWaitNs; lowered only by tests of the failure path through
+// w4_set_wait_limit_ns).  Waits that drain copies before a CTA exits always
+// keep the default.
+constexpr uint64_t kDefaultWaitNs = 200000000ull;   // 200 ms; no legitimate wait comes near it
+// The kernels receive the limit in the low 63 bits of a launch parameter; the
+// top bit, set only by w4_test_stall_first_wait, makes each warp's first wait
+// for a copy target a barrier that nothing completes, so that it runs out.
+constexpr uint64_t kStallFirstWait = 1ull << 63;
+uint64_t wait_limit_ns();
+__host__ __device__ inline uint64_t wait_limit_of(uint64_t w) { return w & ~kStallFirstWait; }
+__host__ __device__ inline bool stalls_first_wait(uint64_t w) { return (w & kStallFirstWait) != 0; }
 // Device address of the library's error word on the current device (nullptr on failure).
 int *device_error_word();
 

@@ -56,7 +56,6 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr int kKB = 64;                      // k per block (one 128-byte swizzle row of bf16)
-constexpr uint64_t kWaitLimitNs = 200000000ull;   // 200 ms; no legitimate wait comes near it
 
 enum : int {
     kErrWaitTma = 0x101, kErrWaitFullA = 0x102, kErrWaitEmptyTma = 0x103, kErrWaitEmptyDeq = 0x104,
@@ -65,16 +64,17 @@ enum : int {
 
 // ---------------------------------------------------------------- PTX ----
 // Wait for the phase of `bar` with the given parity.  Gives up (returns false)
-// when the CTA's abort flag is raised or after kWaitLimitNs, in which case it
+// when the CTA's abort flag is raised or after `limit` ns, in which case it
 // records `code` and raises the abort flag.
-__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int code)
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int code,
+                                         uint64_t limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit) {
             *abort_flag = 1;
             atomicCAS(&g_device_error, 0, code);
             return false;
@@ -87,7 +87,7 @@ __device__ __noinline__ bool wait_drain(uint64_t *bar, uint32_t parity)
 {
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > kDefaultWaitNs) {
             atomicCAS(&g_device_error, 0, kErrDrain);
             return false;
         }
@@ -97,14 +97,15 @@ __device__ __noinline__ bool wait_drain(uint64_t *bar, uint32_t parity)
 
 // Bounded wait until both barriers have completed the phase with the given
 // parity; each round tests both at once (their latencies overlap).
-__device__ __noinline__ bool wait_pair_bounded(uint64_t *a, uint64_t *b, uint32_t parity, volatile int *abort_flag)
+__device__ __noinline__ bool wait_pair_bounded(uint64_t *a, uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                              uint64_t limit)
 {
     const uint64_t t0 = globaltimer();
     while (true) {
         const bool ra = mbar_test(a, parity), rb = mbar_test(b, parity);
         if (ra && rb) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit) {
             *abort_flag = 1;
             atomicCAS(&g_device_error, 0, kErrWaitFullA);
             return false;
@@ -170,7 +171,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                const __grid_constant__ CUtensorMap tmap_y, int y_tma, int M, int N, int K, int group_log2, int asym,
                const uint4 *__restrict__ qweight, const unsigned short *__restrict__ scales,
                const uint32_t *__restrict__ qzeros, __nv_bfloat16 *__restrict__ Y, float *__restrict__ partial,
-               unsigned *__restrict__ counters, int splits, int kb_per_split)
+               unsigned *__restrict__ counters, int splits, int kb_per_split, uint64_t wait_ns)
 {
     using C = TcCfg<BN>;
     constexpr int kStages = C::kStages;
@@ -186,6 +187,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     uint32_t *tmem_slot = (uint32_t *)(done + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
     int *last_flag = (int *)(tmem_slot + 2);
+    uint64_t *stall = (uint64_t *)(tmem_slot + 4);      // a barrier nothing completes (failure tests)
+    const uint64_t limit = wait_limit_of(wait_ns);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * 128, m0 = blockIdx.y * BN, split = blockIdx.z;
@@ -202,6 +205,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
+        mbar_init(stall, 1);
         *abort_flag = 0;
         *last_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -223,7 +227,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % kStages;
                 const uint32_t ph = (i / kStages) & 1;
-                if (!mbar_try_wait(&empty[s], ph ^ 1) && !wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyTma))
+                if (!mbar_try_wait(&empty[s], ph ^ 1) && !wait_bounded(&empty[s], ph ^ 1, abort_flag, kErrWaitEmptyTma, limit))
                     break;
                 mbar_arrive_expect_tx(&full_b[s], C::kStageBytes);
                 tma_load_2d(sB + s * C::kStageBytes, &tmap_x, &full_b[s], (kb_begin + i) * kKB, m0);
@@ -255,7 +259,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 for (int st = 0; st < kStages; ++st) {
                     const int i = i0 + st;
                     if (i >= nkb) break;
-                    if (!ready) ready = wait_pair_bounded(&full_a[st], &full_b[st], ph, abort_flag);
+                    if (!ready) ready = wait_pair_bounded(&full_a[st], &full_b[st], ph, abort_flag, limit);
                     if (!ready) {
                         stop = true;
                         break;
@@ -324,8 +328,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 // (the producer refilled it only after their commit), so its
                 // tensor-memory A columns are free
                 // (the inline try_wait is the usual case: the stage landed long ago)
-                if (!__all_sync(0xffffffffu, mbar_try_wait(&full_b[s], ph) ||
-                                                 wait_bounded(&full_b[s], ph, abort_flag, kErrWaitEmptyDeq))) {
+                // (the first wait of a dequantizing warp targets a barrier that
+                // nothing completes in the failure-path tests)
+                uint64_t *fb = (i == h && stalls_first_wait(wait_ns)) ? stall : &full_b[s];
+                const uint32_t fph = fb == stall ? 0u : ph;
+                if (!__all_sync(0xffffffffu, mbar_try_wait(fb, fph) ||
+                                                 wait_bounded(fb, fph, abort_flag, kErrWaitEmptyDeq, limit))) {
                     ok = false;
                     break;
                 }
@@ -361,7 +369,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         }
 
         // ---- epilogue: accumulator -> Y (or fp32 partials) ----
-        const bool have = __all_sync(0xffffffffu, ok && wait_bounded(done, 0, abort_flag, kErrWaitDone));
+        const bool have = __all_sync(0xffffffffu, ok && wait_bounded(done, 0, abort_flag, kErrWaitDone, limit));
         tc_fence_after();
         constexpr int HALF = BN / 2;                  // columns per warp of a lane quarter
         const int cbeg = h * HALF;
@@ -524,7 +532,7 @@ cudaError_t launch_bn(const CUtensorMap &map, const CUtensorMap &qmap, const CUt
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
     return launch_pdl(gemm_tc_kernel<BN>, grid, dim3(kThreads), smem, stream, map, qmap, ymap, y_tma, M, N, K, glog2,
                       asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros, (__nv_bfloat16 *)Y,
-                      partial, counters, p.splits, p.kb_per_split);
+                      partial, counters, p.splits, p.kb_per_split, wait_limit_ns());
 }
 
 }  // namespace

@@ -67,12 +67,11 @@
 namespace w4 {
 namespace {
 
-constexpr uint64_t kGemvWaitNs = 200000000ull;   // 200 ms; a box lands in microseconds
 constexpr int kErrGemvWait = 0x201, kErrGemvDrain = 0x202;
 
 // Bounded wait for the phase with the given parity of the barrier at shared
-// address `bar`; false after kGemvWaitNs.
-__device__ __noinline__ bool gemv_wait(uint32_t bar, uint32_t parity)
+// address `bar`; false after `limit` ns (a box lands in microseconds).
+__device__ __noinline__ bool gemv_wait(uint32_t bar, uint32_t parity, uint64_t limit = kDefaultWaitNs)
 {
     auto test = [&]() {
         uint32_t ok;
@@ -88,7 +87,7 @@ __device__ __noinline__ bool gemv_wait(uint32_t bar, uint32_t parity)
     if (test()) return true;
     const uint64_t t0 = globaltimer();
     while (!test())
-        if (globaltimer() - t0 > kGemvWaitNs) return false;
+        if (globaltimer() - t0 > limit) return false;
     return true;
 }
 
@@ -114,7 +113,8 @@ struct GemvCfg {
     static constexpr int kChunks = 2 * kBoxes;        // 32-k chunks per lane and stage
     static constexpr int kConstOff = NW * R * kStageBytes;
     static constexpr int kBarOff = kConstOff + NW * kConsts * 16;
-    static constexpr int kBytes = kBarOff + NW * R * 8 + 1024;   // + alignment slack
+    static constexpr int kStallOff = kBarOff + NW * R * 8;      // a barrier nothing completes (failure tests)
+    static constexpr int kBytes = kStallOff + 8 + 1024;          // + alignment slack
     static_assert(SK % 256 == 0 && kCpl >= 1, "stage shape");
     static_assert(32 * 4 * MT * 4 <= R * kStageBytes, "the reduction reuses each warp's stage ring");
 };
@@ -131,7 +131,7 @@ template <int G, int MODE, int MT, int NW, int SK, int R, int MINB, bool EARLY, 
 __global__ void __launch_bounds__(NW * 32, MINB)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
-            __nv_bfloat16 *__restrict__ Y, int *err)
+            __nv_bfloat16 *__restrict__ Y, int *err, uint64_t wait_ns)
 {
     using C = GemvCfg<G, SK, NW, R, MT>;
     extern __shared__ uint8_t smem_raw[];
@@ -150,13 +150,16 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__r
     uint4 *cslot = (uint4 *)(smem + C::kConstOff) + warp * C::kConsts;
     const uint32_t ring_s = smem_u32(ring);
     const uint32_t bar0 = smem_u32(smem + C::kBarOff) + warp * R * 8;
+    const uint32_t stall_bar = smem_u32(smem + C::kStallOff);
+    const uint64_t limit = wait_limit_of(wait_ns);
 
     if (lane == 0) {
         for (int s = 0; s < R; ++s) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8 * s));
+        if (warp == 0) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(stall_bar));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_q) : "memory");
     }
-    __syncwarp();
+    __syncthreads();
     // With EARLY (the caller declared that the kernel before this one on the
     // stream does not write the packed weight), the weight stream starts
     // before the programmatic dependency resolves, overlapping that kernel's
@@ -253,7 +256,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__r
         for (int u = 0; u < C::kCpl; ++u) cslot[lane + 32 * u] = const_word(sv[u], zv[u]);
         if (i + 1 < nsw) load_consts(i + 1);
         __syncwarp();
-        if (!gemv_wait(bar0 + 8 * s, (uint32_t)(i / R) & 1u)) {
+        const bool stall = i == 0 && stalls_first_wait(wait_ns);   // failure-path tests only
+        if (!gemv_wait(stall ? stall_bar : bar0 + 8 * s, stall ? 0u : (uint32_t)(i / R) & 1u, limit)) {
             ok = false;
             break;
         }
@@ -349,7 +353,8 @@ cudaError_t launch_cfg(const CUtensorMap &map, const void *X, int64_t M, int64_t
     const cudaError_t e = set_smem_attr(kern, smem, attr_done);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3((unsigned)blocks), dim3(NW * 32), smem, stream, map, (const __nv_bfloat16 *)X,
-                      (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros, (__nv_bfloat16 *)Y, err);
+                      (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros, (__nv_bfloat16 *)Y, err,
+                      wait_limit_ns());
 }
 
 // Launch shape by tile count (16 channels per tile), chosen from timings on

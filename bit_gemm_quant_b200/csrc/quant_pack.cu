@@ -236,11 +236,11 @@ __device__ __forceinline__ QParams group_params(float a, float mn, float mx, uns
 
 constexpr int kQItemBytes = 32 * 128;              // one item: 32 slices of 64 bf16
 constexpr int kQRingBytes = 8 * 2 * kQItemBytes;   // two items in flight per warp, 8 warps
-constexpr uint64_t kQWaitNs = 200000000ull;        // 200 ms; an item lands in microseconds
 constexpr int kErrQuantWait = 0x401, kErrQuantDrain = 0x402;
 
-// Bounded wait for an item's copy; false after kQWaitNs.
-__device__ __noinline__ bool wait_item(uint32_t bar, uint32_t parity)
+// Bounded wait for an item's copy; false after `limit` ns (an item lands in
+// microseconds).
+__device__ __noinline__ bool wait_item(uint32_t bar, uint32_t parity, uint64_t limit = kDefaultWaitNs)
 {
     uint64_t t0 = 0;
     bool started = false;
@@ -257,7 +257,7 @@ __device__ __noinline__ bool wait_item(uint32_t bar, uint32_t parity)
         if (!started) {
             t0 = globaltimer();
             started = true;
-        } else if (globaltimer() - t0 > kQWaitNs) {
+        } else if (globaltimer() - t0 > limit) {
             return false;
         }
     }
@@ -272,7 +272,7 @@ template <int G, int MODE, bool FOLD, bool TMA>
 __global__ void __launch_bounds__(256, 2)
 quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__restrict__ W, int N, int K,
                   const float *__restrict__ s, int s_staged, uint4 *__restrict__ qweight,
-                  unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros, int *err)
+                  unsigned short *__restrict__ scales, uint32_t *__restrict__ qzeros, int *err, uint64_t wait_ns)
 {
     constexpr int GPL = (G == 32) ? 2 : 1;       // groups per lane: a lane owns 64 consecutive weights
     constexpr int LPG = (G == 128) ? 2 : 1;      // lanes per group
@@ -289,9 +289,12 @@ quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__
     const int wib = (int)(threadIdx.x >> 5);     // warp in block
     const uint32_t ring0 = smem_u32(sbase) + wib * 2 * kQItemBytes;
     const uint32_t bar0 = smem_u32(sbase + kQRingBytes) + wib * 16;
+    const uint32_t stall_bar = smem_u32(sbase + kQRingBytes) + 256 + wib * 8;   // nothing completes it (failure tests)
+    const uint64_t limit = wait_limit_of(wait_ns);
     if (TMA && lane == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0));
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(stall_bar));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_w) : "memory");
     }
@@ -371,7 +374,9 @@ quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__
             // this lane's slice is row `lane` of the box (a lane past the row end
             // reads the next row's slice, or zeros past the matrix: not stored)
             const int sl = j & 1;
-            if (!__all_sync(0xffffffffu, wait_item(bar0 + 8 * sl, (uint32_t)(j >> 1) & 1u))) {
+            const bool stall = j == 0 && stalls_first_wait(wait_ns);   // failure-path tests only
+            if (!__all_sync(0xffffffffu,
+                            wait_item(stall ? stall_bar : bar0 + 8 * sl, stall ? 0u : (uint32_t)(j >> 1) & 1u, limit))) {
                 ok = false;
                 break;
             }
@@ -595,7 +600,7 @@ cudaError_t launch_variant(const CUtensorMap &map, const void *W, int64_t N, int
     if (blocks > cap) blocks = cap;
     return launch_pdl(quant_pack_kernel<G, MODE, FOLD, TMA>, dim3((unsigned)blocks), dim3(threads), smem, stream, map,
                       (const uint32_t *)W, (int)N, (int)K, s, staged, (uint4 *)qweight, (unsigned short *)scales,
-                      qzeros, err);
+                      qzeros, err, wait_limit_ns());
 }
 
 template <int G, int MODE>

@@ -245,6 +245,27 @@ const char *w4_status_string(int status);
 int w4_layout_version(void);
 
 /*
+ * w4_set_wait_limit_ns -- the time after which a kernel's wait for a copy, an
+ * MMA or another warp gives up, records a code (see w4_device_error) and ends
+ * the kernel early; 0 restores the default of 200 ms, far above any
+ * legitimate wait.  This exists to test the failure path: a test lowers the
+ * limit so that a wait runs out, checks the recorded code and that the next
+ * call is correct.  Waits that let a kernel's own copies and MMAs finish
+ * before it exits always keep the default.  Process-wide; read at each launch.
+ */
+void w4_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * w4_test_stall_first_wait -- for tests of the failure path only: while `on`
+ * is nonzero, each warp's first wait for a copy (in w4_quant_pack and
+ * w4a16_gemm) targets a barrier that nothing completes, so that it runs out
+ * after the limit set by w4_set_wait_limit_ns and the kernel takes its failure
+ * path; the copies it issued still land (they are drained with the default
+ * limit).  0 (the default) turns it off.  Process-wide; read at each launch.
+ */
+void w4_test_stall_first_wait(int on);
+
+/*
  * w4_device_error -- read and clear the library's device-side error word.
  * Kernels that wait on barriers give every wait an iteration limit; a wait
  * that runs out records a nonzero code here and the kernel returns early

@@ -138,9 +138,13 @@ def test_grid_point_within_half_a_step(mode):
 def test_scene4_output_error_down_weight_error_up():
     # INT4 g=64 on calibration features with low-rank correlation: the printed
     # result is a 2.85x smaller output error with a larger weight error.
+    # The fixture bounds the oracle: its output-error ratio RTN / GPTQ must be at
+    # least the printed ratio, and its weight error must move in the printed
+    # direction (the setups differ, so only the direction and the size of the
+    # gain are compared).
     fx = golden("gptq_scene4.json")["printed"]
-    assert fx["gptq"]["output_rel_l2"] < fx["rtn"]["output_rel_l2"] / 2
-    assert fx["gptq"]["weight_rel_l2"] > fx["rtn"]["weight_rel_l2"]
+    printed_ratio = fx["rtn"]["output_rel_l2"] / fx["gptq"]["output_rel_l2"]
+    weight_error_rises = fx["gptq"]["weight_rel_l2"] > fx["rtn"]["weight_rel_l2"]
     N, K, M, g = 64, 256, 512, 64
     W = bits(np.random.default_rng(7).standard_normal((N, K)))
     X = correlated_calibration(8, M, K, rank=16, noise=0.02)
@@ -152,5 +156,5 @@ def test_scene4_output_error_down_weight_error_up():
     werr = lambda Wh: np.linalg.norm(Wh - w) / np.linalg.norm(w)
     out_g = gptq.output_error(W, What_g, X)
     out_r = gptq.output_error(W, What_r, X)
-    assert out_g < out_r / 2
-    assert werr(What_g) > werr(What_r)
+    assert out_r / out_g >= printed_ratio
+    assert (werr(What_g) > werr(What_r)) == weight_error_rises

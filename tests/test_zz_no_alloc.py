@@ -1,8 +1,9 @@
 """w4a16_gemm_noalloc: the entry point for callers that cannot allocate
-device memory.  It must give the same product as w4a16_gemm (which takes a
-caller-allocated workspace) on a split-K shape, on consecutive calls that
-share the library's fixed scratch array, and must reject shapes whose scratch
-need exceeds that array before launching anything.
+device memory.  It must give the product the CPU oracle defines (and the same
+product as w4a16_gemm, which takes a caller-allocated workspace) on a split-K
+shape, on consecutive calls that share the library's fixed scratch array, and
+must reject shapes whose scratch need exceeds that array before launching
+anything.
 
 This file is collected last so that it runs both after every other test and,
 alone, in a fresh process."""
@@ -12,9 +13,10 @@ import re
 import numpy as np
 import pytest
 
+import oracle
 from bit_gemm_quant_b200 import synth
 from conftest import ROOT
-from parity import assert_y_close, dev_bf16, host_bf16_as_f64
+from parity import THREADS, assert_y_close, dev_bf16, host_bf16_as_f64
 
 SYM, ASYM = 0, 1
 
@@ -61,6 +63,9 @@ def test_noalloc_matches_workspace_entry_point_twice(w4, M, N, K, g, mode):
     q, sc, z = w4.quant_pack(dev_bf16(W), g, mode)
     Xd = dev_bf16(X)
     Y_ws = host_bf16_as_f64(w4.gemm(Xd, q, sc, z, g, mode))   # caller-allocated, zeroed workspace
+    oracle.build()
+    oq, osc, oz = oracle.quant_pack(W, g, mode, threads=THREADS)
+    Y_ref = oracle.w4a16_reference(X, oq, osc, oz, K, g, mode, threads=THREADS)
     stream = torch.cuda.current_stream()
     for call in range(2):                                       # the second call reuses the scratch
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -72,5 +77,6 @@ def test_noalloc_matches_workspace_entry_point_twice(w4, M, N, K, g, mode):
         torch.cuda.synchronize()
         Yn = host_bf16_as_f64(Y)
         assert np.isfinite(Yn).all(), "call %d left outputs unwritten" % call
-        assert_y_close(Yn, Y_ws, what="noalloc call %d" % call)
+        assert_y_close(Yn, Y_ref, what="noalloc call %d against the oracle" % call)
+        assert_y_close(Yn, Y_ws, what="noalloc call %d against w4a16_gemm" % call)
     assert w4.w4_device_error() == 0
