@@ -19,6 +19,7 @@ SYM, ASYM = 0, 1
 WEIGHTS_STATIC = 0x100
 NVFP4, MXFP4 = 0, 1
 FP4_BLOCK = {NVFP4: 16, MXFP4: 32}
+MX_SCALES_ROWS, MX_SCALES_MMA = 0, 1
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA = 0, 1, 2, 3
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
@@ -53,6 +54,14 @@ def lib() -> ctypes.CDLL:
         L.w4_awq_search.restype = I
         L.w4_fp4_quant.argtypes = [P, I64, I64, I, P, P, P]
         L.w4_fp4_quant.restype = I
+        L.w4_mxfp8_quant.argtypes = [P, I64, I64, P, P, I, P]
+        L.w4_mxfp8_quant.restype = I
+        L.w4_mx_scale_layout.argtypes = [P, I64, I64, P, P]
+        L.w4_mx_scale_layout.restype = I
+        L.w4_mx_workspace_bytes.argtypes = [I64, I64, I64]
+        L.w4_mx_workspace_bytes.restype = SZ
+        L.w4_mx_gemm.argtypes = [P, P, I64, I64, I64, P, P, P, P, SZ, P]
+        L.w4_mx_gemm.restype = I
         L.w4_status_string.argtypes = [I]
         L.w4_status_string.restype = ctypes.c_char_p
         L.w4_layout_version.argtypes = []
@@ -98,6 +107,22 @@ def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, wor
 
 def w4_fp4_quant(W, N, K, kind, codes, scales, stream) -> int:
     return lib().w4_fp4_quant(W, N, K, kind, codes, scales, stream)
+
+
+def w4_mxfp8_quant(X, M, K, codes, scales, scale_layout, stream) -> int:
+    return lib().w4_mxfp8_quant(X, M, K, codes, scales, scale_layout, stream)
+
+
+def w4_mx_scale_layout(src, R, K, dst, stream) -> int:
+    return lib().w4_mx_scale_layout(src, R, K, dst, stream)
+
+
+def w4_mx_workspace_bytes(M, N, K) -> int:
+    return int(lib().w4_mx_workspace_bytes(M, N, K))
+
+
+def w4_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, workspace, workspace_bytes, stream) -> int:
+    return lib().w4_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, workspace, workspace_bytes, stream)
 
 
 def w4_status_string(status: int) -> str:
@@ -233,3 +258,58 @@ def fp4_quant(W, kind: int = NVFP4, stream=None, out=None):
     if st != W4_OK:
         raise W4Error(st, "w4_fp4_quant")
     return codes, scales
+
+
+def mx_scale_bytes(R: int, K: int) -> int:
+    """Bytes of E8M0 scales for R rows x K columns in the tensor-core layout."""
+    return (R + 127) // 128 * 128 * (K // 32)
+
+
+def mxfp8_quant(X, scale_layout: int = MX_SCALES_MMA, stream=None, out=None):
+    """MXFP8 quantization of a bf16 CUDA tensor X[M,K].
+    Returns (codes uint8 [M, K], scales uint8: [M, K/32] for MX_SCALES_ROWS,
+    flat [mx_scale_bytes(M, K)] for MX_SCALES_MMA)."""
+    import torch
+    M, K = X.shape
+    if out is None:
+        codes = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+        if scale_layout == MX_SCALES_ROWS:
+            scales = torch.empty((M, max(K // 32, 1)), dtype=torch.uint8, device=X.device)
+        else:
+            scales = torch.empty(max(mx_scale_bytes(M, K), 1), dtype=torch.uint8, device=X.device)
+    else:
+        codes, scales = out
+    st = w4_mxfp8_quant(_ptr(X), M, K, _ptr(codes), _ptr(scales), scale_layout, _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_mxfp8_quant")
+    return codes, scales
+
+
+def mx_scale_layout(scales_rows, K: int, stream=None, out=None):
+    """E8M0 scales uint8 [R, K/32] (CUDA) to the tensor-core layout (flat uint8)."""
+    import torch
+    R = scales_rows.shape[0]
+    dst = out if out is not None else torch.empty(mx_scale_bytes(R, K), dtype=torch.uint8,
+                                                  device=scales_rows.device)
+    st = w4_mx_scale_layout(_ptr(scales_rows), R, K, _ptr(dst), _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_mx_scale_layout")
+    return dst
+
+
+def mx_gemm(x_codes, x_scales, w_codes, w_scales, workspace=None, out=None, stream=None):
+    """Y[M,N] bf16 = X^ . W^^T from MXFP8 activations (codes [M,K], tensor-core
+    layout scales) and MXFP4 weights (codes [N,K/2], tensor-core layout scales)."""
+    import torch
+    M, K = x_codes.shape
+    N = w_codes.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device)
+    need = w4_mx_workspace_bytes(M, N, K)
+    if need and workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x_codes.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = w4_mx_gemm(_ptr(x_codes), _ptr(x_scales), M, N, K, _ptr(w_codes), _ptr(w_scales), _ptr(Y), _ptr(workspace),
+                    wbytes, _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_mx_gemm")
+    return Y

@@ -82,6 +82,65 @@ w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *c
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+w4_status w4_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales, int scale_layout,
+                         w4_stream_t stream)
+{
+    if (!X || !codes || !scales) return W4_ERR_INVALID_ARG;
+    if (scale_layout != W4_MX_SCALES_ROWS && scale_layout != W4_MX_SCALES_MMA) return W4_ERR_INVALID_ARG;
+    if (M < 1 || K < 32 || K % 32 != 0 || !fits(M, K)) return W4_ERR_INVALID_ARG;
+    if (scale_layout == W4_MX_SCALES_MMA && K % 128 != 0) return W4_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(codes, 16)) return W4_ERR_INVALID_ARG;
+    if (scale_layout == W4_MX_SCALES_MMA && !aligned(scales, 16)) return W4_ERR_INVALID_ARG;
+    if (!fits(w4::mx_padded_rows(M), K)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e = w4::launch_mxfp8_quant(X, M, K, codes, scales, scale_layout, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_mx_scale_layout(const uint8_t *src, int64_t R, int64_t K, uint8_t *dst, w4_stream_t stream)
+{
+    if (!src || !dst) return W4_ERR_INVALID_ARG;
+    if (R < 1 || K < 128 || K % 128 != 0 || !fits(R, K) || !fits(w4::mx_padded_rows(R), K)) return W4_ERR_INVALID_ARG;
+    if (!aligned(src, 4) || !aligned(dst, 16)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e = w4::launch_mx_scale_layout(src, R, K, dst, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+namespace {
+bool mx_shape_ok(int64_t M, int64_t N, int64_t K)
+{
+    return M >= 1 && N >= 1 && K >= 128 && K % 128 == 0 && fits(M, K) && fits(N, K) && fits(M, N);
+}
+// 32-bit indices in the kernel (rows, columns, split partial offsets use size_t)
+bool mx_shape_supported(int64_t M, int64_t N, int64_t K)
+{
+    return M <= INT32_MAX - 256 && N <= INT32_MAX - 128 && K <= INT32_MAX && M * K <= (int64_t)1 << 40 &&
+           N * K <= (int64_t)1 << 40;
+}
+}  // namespace
+
+size_t w4_mx_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (!mx_shape_ok(M, N, K) || !mx_shape_supported(M, N, K)) return 0;
+    return w4::mx_workspace_bytes(M, N, K);
+}
+
+w4_status w4_mx_gemm(const uint8_t *x_codes, const uint8_t *x_scales, int64_t M, int64_t N, int64_t K,
+                     const uint8_t *w_codes, const uint8_t *w_scales, void *Y, void *workspace,
+                     size_t workspace_bytes, w4_stream_t stream)
+{
+    if (!x_codes || !x_scales || !w_codes || !w_scales || !Y) return W4_ERR_INVALID_ARG;
+    if (!mx_shape_ok(M, N, K)) return W4_ERR_INVALID_ARG;
+    if (!aligned(x_codes, 16) || !aligned(x_scales, 16) || !aligned(w_codes, 32) || !aligned(w_scales, 16) ||
+        !aligned(Y, 2))
+        return W4_ERR_INVALID_ARG;
+    if (!mx_shape_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
+    const size_t need = w4::mx_workspace_bytes(M, N, K);
+    if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256)))) return W4_ERR_INVALID_ARG;
+    const cudaError_t e =
+        w4::launch_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, workspace, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group)
 {
     (void)group;

@@ -90,6 +90,14 @@ cudaError_t set_smem_attr(Kern kern, int bytes, std::atomic<bool> (&done)[kMaxDe
 }
 cudaError_t launch_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                              cudaStream_t stream);
+// MX activations, the tensor-core scale layout and the block-scaled product
+int64_t mx_padded_rows(int64_t R);
+cudaError_t launch_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales, int layout,
+                               cudaStream_t stream);
+cudaError_t launch_mx_scale_layout(const uint8_t *src, int64_t R, int64_t K, uint8_t *dst, cudaStream_t stream);
+size_t mx_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_mx_gemm(const uint8_t *x_codes, const uint8_t *x_sf, int64_t M, int64_t N, int64_t K,
+                           const uint8_t *w_codes, const uint8_t *w_sf, void *Y, void *ws, cudaStream_t stream);
 size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
 // byte range of the split-K tile counters inside that workspace (0 bytes if none)
 void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size_t *bytes);

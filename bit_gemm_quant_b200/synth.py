@@ -24,6 +24,8 @@ SmoothQuant sections of the pages):
               the smoothing fold with s = act^0.5/mean(act^0.5),
               act = |N(0,1)| with 1% of channels x20.
   decodequant the decode workload's three weights, quantized (no product).
+  mxdecode    the decode workload's layers (same seeds and distributions) for
+              the block-scaled product: MXFP4 weights, MXFP8 activations.
 
 "p% outlier channels" are the first round(p*K) entries of a seeded
 permutation of 0..K-1; weight columns and activation channels are drawn
@@ -145,6 +147,9 @@ def workload(name: str) -> list[Problem]:
         # the decode layers' weights (same seeds as the decode workload), quantized
         return [Problem("decode_N%d" % N, 0, N, 4096, 128, ASYM, 0.02, (0.01, 5.0), seed=1)
                 for N in (4096, 11008, 12288)]
+    if name == "mxdecode":
+        return [Problem("mxdecode_N%d" % N, 1, N, 4096, 128, ASYM, 0.02, (0.01, 5.0), (0.01, 40.0), seed=1)
+                for N in (4096, 11008, 12288)]
     if name == "quantizer":
         probs = []
         for g in (32, 64, 128):
@@ -156,4 +161,4 @@ def workload(name: str) -> list[Problem]:
     raise KeyError(name)
 
 
-WORKLOADS = ("tiny", "decode", "smallbatch", "prefill", "quantizer", "decodequant")
+WORKLOADS = ("tiny", "decode", "smallbatch", "prefill", "quantizer", "decodequant", "mxdecode")

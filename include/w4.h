@@ -238,6 +238,90 @@ w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int64_t K, con
 w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                        w4_stream_t stream);
 
+/*
+ * MX scale layouts (for the E8M0 scales of w4_mxfp8_quant, w4_mx_scale_layout
+ * and w4_mx_gemm; R rows, K columns, one scale per 32-element block kb):
+ *   W4_MX_SCALES_ROWS  uint8 [R][K/32], byte r * (K/32) + kb.
+ *   W4_MX_SCALES_MMA   the tensor-core layout: ceil(R/128) bands of 128 rows,
+ *                      each band K/128 atoms of 512 bytes in k order; the
+ *                      scale of (r, kb) is the byte at
+ *                        ((r/128) * (K/128) + kb/4) * 512
+ *                          + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4.
+ *                      Size ceil(R/128) * 128 * (K/32) bytes; the bytes of
+ *                      rows R.. of the last band are written as 0.
+ */
+#define W4_MX_SCALES_ROWS 0
+#define W4_MX_SCALES_MMA 1
+
+/*
+ * w4_mxfp8_quant -- MXFP8 quantization of bf16 activations.
+ *   (page 3 section 4.3: activations kept at FP8 beside FP4 weights, one
+ *    E8M0 scale per block of 32 elements; page 5 section 2.1 and page 3
+ *    section 4.1: the E4M3 format)
+ *   Exact semantics, per block of 32 consecutive elements of a row:
+ *     amax = max |x| over the block
+ *     e    = clamp(floor(log2 amax) - 8, -127, 127) (-127 for an all-zero
+ *            block); scale code = e + 127 (E8M0); s = 2^e
+ *     code = e4m3_rne_satfinite(fl32(x / s)): round to nearest even, finite
+ *            magnitudes above 448 giving 448 (a block's largest elements clip
+ *            when amax lies in [1.75, 2) * 2^(e+8)); the sign follows x / s
+ *     x^   = e4m3(code) * s (exact)
+ *   X        bf16 [M][K], finite, 16-byte aligned.
+ *   M, K     M >= 1, K >= 32, K % 32 == 0; K % 128 == 0 for W4_MX_SCALES_MMA.
+ *   codes    out, uint8 [M][K] E4M3 codes, 16-byte aligned.
+ *   scales   out, E8M0 codes in `scale_layout` (W4_MX_SCALES_ROWS: [M][K/32];
+ *            W4_MX_SCALES_MMA: see above, 16-byte aligned).
+ * Every output byte is written; outputs must not overlap inputs.
+ * Errors: W4_ERR_INVALID_ARG for a NULL or misaligned pointer, a bad size or
+ * layout; W4_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ */
+w4_status w4_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales, int scale_layout,
+                         w4_stream_t stream);
+
+/*
+ * w4_mx_scale_layout -- copy E8M0 scales from W4_MX_SCALES_ROWS to
+ * W4_MX_SCALES_MMA (a permutation of bytes, plus the zero rows that pad the
+ * last band).  Used once per weight: w4_fp4_quant(W4_MXFP4) writes rows.
+ *   src      uint8 [R][K/32], 4-byte aligned.
+ *   R, K     R >= 1, K >= 128, K % 128 == 0.
+ *   dst      out, ceil(R/128) * 128 * (K/32) bytes, 16-byte aligned.
+ * Errors as for w4_mxfp8_quant.
+ */
+w4_status w4_mx_scale_layout(const uint8_t *src, int64_t R, int64_t K, uint8_t *dst, w4_stream_t stream);
+
+/*
+ * w4_mx_workspace_bytes -- device scratch that w4_mx_gemm needs for this
+ * shape (split-K partial sums and tile counters), 0 if none.  Same contract
+ * as w4a16_workspace_bytes: zero-filled before its first use with a shape,
+ * left zero-filled by every successful call.
+ */
+size_t w4_mx_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * w4_mx_gemm -- Y = X^ . W^^T for MXFP8 activations and MXFP4 weights on the
+ * block-scaled tensor cores (page 3 section 4.3: FP4 weights times FP8
+ * activations, E8M0 scales per 32; page 2, the Blackwell FP4 paragraph: the
+ * block-scaled format feeds the tensor cores directly).
+ *   Y[m][n] = bf16_rne(sum_k x^[m][k] * w^[n][k]) with x^ from
+ *   w4_mxfp8_quant, w^ from w4_fp4_quant(W4_MXFP4) (w^ = e2m1(code) * 2^e),
+ *   accumulated by the tensor cores in fp32 (the summation order is the
+ *   hardware's).
+ *   x_codes  uint8 [M][K] E4M3 codes, 16-byte aligned.
+ *   x_scales E8M0, W4_MX_SCALES_MMA layout for M rows, 16-byte aligned.
+ *   M, N, K  M >= 1, N >= 1, K >= 128, K % 128 == 0.
+ *   w_codes  uint8 [N][K/2] MXFP4 codes (w4_fp4_quant layout), 32-byte aligned.
+ *   w_scales E8M0, W4_MX_SCALES_MMA layout for N rows, 16-byte aligned.
+ *   Y        out, bf16 [M][N], 2-byte aligned.
+ *   workspace, workspace_bytes: w4_mx_workspace_bytes(M, N, K) bytes,
+ *            256-byte aligned (may be NULL when that is 0).
+ * Errors: W4_ERR_INVALID_ARG for a NULL or misaligned pointer, a bad size or
+ * a short workspace; W4_ERR_UNSUPPORTED for shapes past 32-bit indexing;
+ * W4_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ */
+w4_status w4_mx_gemm(const uint8_t *x_codes, const uint8_t *x_scales, int64_t M, int64_t N, int64_t K,
+                     const uint8_t *w_codes, const uint8_t *w_scales, void *Y, void *workspace,
+                     size_t workspace_bytes, w4_stream_t stream);
+
 /* Text for a status code; never NULL. */
 const char *w4_status_string(int status);
 
@@ -257,8 +341,8 @@ void w4_set_wait_limit_ns(uint64_t ns);
 
 /*
  * w4_test_stall_first_wait -- for tests of the failure path only: while `on`
- * is nonzero, each warp's first wait for a copy (in w4_quant_pack and
- * w4a16_gemm) targets a barrier that nothing completes, so that it runs out
+ * is nonzero, each warp's first wait for a copy (in w4_quant_pack,
+ * w4a16_gemm and w4_mx_gemm) targets a barrier that nothing completes, so that it runs out
  * after the limit set by w4_set_wait_limit_ns and the kernel takes its failure
  * path; the copies it issued still land (they are drained with the default
  * limit).  0 (the default) turns it off.  Process-wide; read at each launch.

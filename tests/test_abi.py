@@ -197,3 +197,58 @@ def test_noalloc_rejects_an_unsupported_shape_before_enqueuing_anything(w4):
     assert st == U
     need = w4.w4a16_workspace_bytes(64, 128, 1 << 26, 128)
     assert mm(w4, M=64, N=128, K=1 << 26, ws=FAKE, wsb=need) == U   # w4a16_gemm agrees
+
+
+def mq(w4, X=FAKE, M=4, K=256, c=FAKE, sc=FAKE, layout=1):
+    return w4.w4_mxfp8_quant(P(X) if X else None, M, K, P(c) if c else None, P(sc) if sc else None, layout, None)
+
+
+def test_mxfp8_quant_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    assert mq(w4, X=0) == E and mq(w4, c=0) == E and mq(w4, sc=0) == E
+    assert mq(w4, layout=2) == E and mq(w4, layout=-1) == E
+    assert mq(w4, M=0) == E                      # empty input
+    assert mq(w4, K=0) == E and mq(w4, K=16) == E and mq(w4, K=48) == E
+    assert mq(w4, K=96, layout=1) == E           # the tensor-core layout needs K % 128 == 0
+    assert mq(w4, X=FAKE + 2) == E               # 16-byte loads
+    assert mq(w4, c=FAKE + 8) == E
+    assert mq(w4, sc=FAKE + 4, layout=1) == E    # bulk-copied atoms need 16-byte alignment
+    assert mq(w4, M=1 << 40, K=1 << 30) == E     # M*K overflows int64
+
+
+def test_mx_scale_layout_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    f = lambda src=FAKE, R=256, K=512, dst=FAKE: w4.w4_mx_scale_layout(P(src) if src else None, R, K,
+                                                                      P(dst) if dst else None, None)
+    assert f(src=0) == E and f(dst=0) == E
+    assert f(R=0) == E and f(K=64) == E and f(K=160) == E
+    assert f(src=FAKE + 2) == E and f(dst=FAKE + 8) == E
+
+
+def mxg(w4, xc=FAKE, xs=FAKE, M=1, N=256, K=512, wc=FAKE, wsf=FAKE, Y=FAKE, ws=None, wsb=0):
+    return w4.w4_mx_gemm(P(xc) if xc else None, P(xs) if xs else None, M, N, K, P(wc) if wc else None,
+                         P(wsf) if wsf else None, P(Y) if Y else None, P(ws) if ws else None, wsb, None)
+
+
+def test_mx_gemm_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    for kw in ("xc", "xs", "wc", "wsf", "Y"):
+        assert mxg(w4, **{kw: 0}) == E
+    assert mxg(w4, M=0) == E and mxg(w4, N=0) == E
+    assert mxg(w4, K=64) == E and mxg(w4, K=192) == E        # whole 128-wide k-stages only
+    assert mxg(w4, wc=FAKE + 16) == E                         # the FP4 tensor map wants 32-byte alignment
+    assert mxg(w4, xc=FAKE + 8) == E and mxg(w4, xs=FAKE + 8) == E and mxg(w4, wsf=FAKE + 4) == E
+    assert mxg(w4, Y=FAKE + 1) == E
+    # a shape that splits k needs its workspace
+    need = w4.w4_mx_workspace_bytes(1, 4096, 4096)
+    assert need > 0
+    assert mxg(w4, N=4096, K=4096) == E
+    assert mxg(w4, N=4096, K=4096, ws=FAKE, wsb=need - 1) == E
+    assert mxg(w4, N=4096, K=4096, ws=FAKE + 64, wsb=need) == E
+
+
+def test_mx_workspace_query_is_host_only(w4):
+    assert w4.w4_mx_workspace_bytes(1, 4096, 4096) > 0        # 32 tiles: k is split
+    assert w4.w4_mx_workspace_bytes(1, 28672, 8192) == 0      # 224 tiles fill the SMs
+    assert w4.w4_mx_workspace_bytes(1, 4096, 4000) == 0       # malformed
+    assert w4.w4_mx_workspace_bytes(0, 4096, 4096) == 0
