@@ -20,6 +20,8 @@ The quantizer workloads time the quantization itself.
   decodequant       w4_quant_pack of the decode weights (K=4096, N in {4096, 11008, 12288}, asym g=128)
   awq               the AWQ scale search over W[4096, 4096] with 128 calibration rows
   fp4quant          W[28672, 8192] to NVFP4 and to MXFP4: 2 x w4_fp4_quant per step
+  mxdecode          the decode layers with MXFP4 weights and MXFP8 activations: per layer
+                    w4_mxfp8_quant + w4_mx_gemm (block-scaled tcgen05); value = algorithmic GB/s
 
 The K timed steps are captured in one CUDA graph (kernel nodes only) and
 replayed once between CUDA events on the launching stream.  Inputs rotate over
@@ -60,7 +62,7 @@ from bit_gemm_quant_b200 import roofline, synth  # noqa: E402
 
 METRIC = "W4A16 g128 GEMV HBM GB/s (% peak); GEMM TFLOPS (% peak); quant-pack GB/s"
 KERNEL_SOURCES = {"w4_quant_pack": "quant_pack.cu", "w4a16_gemv": "gemv.cu", "w4a16_gemm_tc": "gemm_tc.cu",
-                  "w4_fp4_quant": "fp4_quant.cu"}
+                  "w4_fp4_quant": "fp4_quant.cu", "w4_mx_gemm": "mx_gemm.cu", "w4_mxfp8_quant": "mx_quant.cu"}
 THROTTLE_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -70,7 +72,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["w4", "reference"], default="w4")
-    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "decodequant", "awq", "fp4quant"],
+    ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "decodequant", "awq", "fp4quant",
+                                               "mxdecode"],
                     default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -131,6 +134,9 @@ WORKLOAD_DESC = {
                    "step = 3 w4_quant_pack",
     "fp4quant": "block-scaled FP4 weight quantization: W[28672,8192] bf16 to NVFP4 (E2M1, E4M3 scale per 16) and "
                 "to MXFP4 (E2M1, E8M0 scale per 32); step = 2 w4_fp4_quant",
+    "mxdecode": "MX decode: M=1, K=4096, N in {4096,11008,12288}, MXFP4 weights (E2M1, E8M0 scale per 32) x MXFP8 "
+                "activations (E4M3, E8M0 scale per 32); step = per layer w4_mxfp8_quant + w4_mx_gemm "
+                "(tcgen05.mma kind::mxf8f6f4, W4_WEIGHTS_STATIC), weights quantized once before timing",
 }
 
 
@@ -702,6 +708,8 @@ def run_reference(args, rank, world):
         return run_reference_awq(args, world)
     if args.workload == "fp4quant":
         return run_reference_fp4(args, world)
+    if args.workload in MX_WORKLOADS:
+        return run_reference_mx(args, world)
     plist = problems_for(args.workload)
     keys = list(dict.fromkeys(k for k, _ in plist))
     first = {k: p for k, p in reversed(plist)}
@@ -1117,6 +1125,300 @@ def fp4_e2e(w4, torch, device, host_W, steps):
             "steps": steps}
 
 
+# ------------------------------------------------------------ MX product --
+
+MX_WORKLOADS = ("mxdecode",)
+MXFP4_KIND = 1
+
+
+def mx_step_bytes(probs) -> int:
+    return sum(roofline.mxfp8_quant_bytes(p.M, p.K) + roofline.mx_gemm_bytes(p.M, p.N, p.K) for p in probs)
+
+
+def graph_launch_ms(torch, device, fns, KL, replays=5):
+    """Median and min per-launch time of a CUDA graph of KL launches cycling
+    over fns, between CUDA events on the graph's stream."""
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(device)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cs):
+        for i in range(KL):
+            fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    per = []
+    for _ in range(replays):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(cs):
+            e0.record(cs)
+            g.replay()
+            e1.record(cs)
+        e1.synchronize()
+        per.append(e0.elapsed_time(e1) / KL)
+    del g
+    return statistics.median(per), min(per)
+
+
+def run_mx(args, rank, world, local_rank):
+    """The decode layers with MXFP4 weights and MXFP8 activations (page 3
+    section 4.3): per layer, the activation quantization and the block-scaled
+    tensor-core product.  The weights are quantized and their scales laid out
+    once before timing (model state); each step reads them from one of
+    several copies whose reuse distance exceeds 3x L2."""
+    import torch
+    import bit_gemm_quant_b200 as w4
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    w4.lib()
+    pk = roofline.peaks(ROOT)
+    probs = synth.workload(args.workload)
+    rank_seed = 1000 * rank
+    host_W = [synth.weights(p.seed + rank_seed, p.N, p.K, p.w_std, *p.w_outlier) for p in probs]
+    host_X = [synth.activations(p.seed + rank_seed, p.M, p.K, *p.x_outlier) for p in probs]
+    dev = lambda bits: torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16)
+
+    state = []
+    for p, hw in zip(probs, host_W):
+        Wd = dev(hw)
+        c, s_rows = w4.fp4_quant(Wd, w4.MXFP4)
+        state.append((c, w4.mx_scale_layout(s_rows, p.K)))
+        del Wd, s_rows
+    wbytes = sum(c.numel() + s.numel() for c, s in state)
+    copies = max(2, -(-3 * (126 << 20) // wbytes) + 1)
+    pools = [[st] + [(st[0].clone(), st[1].clone()) for _ in range(copies - 1)] for st in state]
+    X_d = [dev(hx) for hx in host_X]
+    xq = [w4.mxfp8_quant(x, w4.MX_SCALES_MMA) for x in X_d]
+    Y_d = [torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device) for p in probs]
+    torch.cuda.synchronize()
+
+    def layer(i, copy):
+        c, s = pools[i][copy % copies]
+        w4.mxfp8_quant(X_d[i], w4.MX_SCALES_MMA, out=xq[i])
+        w4.mx_gemm(xq[i][0], xq[i][1], c, s, out=Y_d[i], weights_static=True)
+
+    def step(si):
+        for i in range(len(probs)):
+            layer(i, si)
+
+    for si in range(max(3, args.warmup)):
+        step(si)
+    torch.cuda.synchronize()
+    K_steps = args.steps
+    graph = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(device)
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cs):
+        for si in range(K_steps):
+            step(si)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(smi_gpu_id(local_rank))
+    sampler.start()
+    sampler.mark_begin()
+    t_end = time.time() + 1.5
+    replays = 0
+    while time.time() < t_end or replays < 2:
+        graph.replay()
+        replays += 1
+        torch.cuda.synchronize()
+
+    def timed():
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(cs):
+            e0.record(cs)
+            graph.replay()
+            e1.record(cs)
+        e1.synchronize()
+        barrier()
+        return e0.elapsed_time(e1)
+
+    local_ms = timed()
+    sampler.mark_end()
+    clocks = sampler.stop()
+    if any(r in clocks.get("reasons", []) for r in THROTTLE_REASONS):
+        sampler = ClockSampler(sampler.gpu_id)
+        sampler.start()
+        sampler.mark_begin()
+        local_ms = timed()
+        sampler.mark_end()
+        clocks = sampler.stop()
+        clocks["remeasured"] = True
+    del graph
+
+    # each kernel of each layer alone (the product over the rotating weight
+    # copies, with W4_WEIGHTS_STATIC as in the step and without it)
+    KL = max(K_steps, 100)
+    kernels = {}
+    gemm_times = []
+    gemm_plain = []
+    for i, p in enumerate(probs):
+        nb = roofline.mx_gemm_bytes(p.M, p.N, p.K)
+        for static in (True, False):
+            fns = [(lambda i=i, j=j, st=static: w4.mx_gemm(xq[i][0], xq[i][1], pools[i][j][0], pools[i][j][1],
+                                                          out=Y_d[i], weights_static=st)) for j in range(copies)]
+            avg, mn = graph_launch_ms(torch, device, fns, KL)
+            (gemm_times if static else gemm_plain).append((nb, avg))
+            kernels["w4_mx_gemm%s[%s]" % ("" if static else "_plain", p.name)] = {
+                "launches": KL * 5, "avg_us": round(avg * 1e3, 3), "min_us": round(mn * 1e3, 3), "bytes": nb,
+                "gbs": round(nb / (avg * 1e-3) / 1e9, 1), "hbm_frac": round(nb / (avg * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                "weights_static": static}
+        avg, mn = graph_launch_ms(torch, device, [lambda i=i: w4.mxfp8_quant(X_d[i], w4.MX_SCALES_MMA, out=xq[i])], KL)
+        nb = roofline.mxfp8_quant_bytes(p.M, p.K)
+        kernels["w4_mxfp8_quant[%s]" % p.name] = {
+            "launches": KL * 5, "avg_us": round(avg * 1e3, 3), "min_us": round(mn * 1e3, 3), "bytes": nb,
+            "gbs": round(nb / (avg * 1e-3) / 1e9, 1)}
+    torch.cuda.synchronize()
+
+    work = K_steps * mx_step_bytes(probs)
+    max_ms, total = aggregate(local_ms, work, device)
+    value = total / (max_ms * 1e-3) / 1e9
+    per_launch = sum(nb for nb, _ in gemm_times) / len(gemm_times)
+    avg_ms = sum(t for _, t in gemm_times) / len(gemm_times)
+    achieved = per_launch / (avg_ms * 1e-3) / 1e9
+    traffic = traffic_table()
+    tr = [traffic.get(("w4_mx_gemm", p.name)) for p in probs]
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4),
+            "traffic": (sum(tr) / len(tr)) if all(t is not None for t in tr) else None,
+            "kernel": "w4_mx_gemm", "algorithmic_per_launch": per_launch, "weights_static": True,
+            "frac_plain": round(per_launch / (sum(t for _, t in gemm_plain) / len(gemm_plain) * 1e-3) / 1e9
+                                / pk["hbm_gbs"], 4),
+            "peak_source": "%s (%s)" % (pk["source"], "MEASURED_PEAKS.json" if pk["source"] == "measured"
+                                        else "recipe")}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = mx_e2e(w4, torch, device, probs, state, host_X, min(K_steps, 10))
+        e_ms, e_work = aggregate(e2e["ms"], e2e["work"], device)
+        e2e = {"value": round(e_work / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
+               "what": e2e["what"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_mx(probs, host_W, host_X, args.cpu_budget)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K_steps,
+            "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / K_steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e4m3 (E8M0 scales), fp32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_DESC[args.workload],
+                       "l2": "every product reads its weight from one of %d copies (reuse distance > 3x L2)" % copies,
+                       "timing": "K steps captured in one CUDA graph, replayed between CUDA events on the launching "
+                                 "stream after %d untimed replays; max over ranks; per-kernel durations: median (and "
+                                 "min) over 5 replays of a graph of max(K, 100) launches of that kernel alone" % replays,
+                       "parallelism": "replicas (dp%d), no data-path collective" % world},
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": K_steps * 2 * len(probs) * world, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def mx_e2e(w4, torch, device, probs, state, host_X, steps):
+    """Through the tensor API with pinned host buffers, all timed: per layer the
+    host->device copy of X, its MXFP8 quantization, the product and the
+    device->host copy of Y (the quantized weights resident)."""
+    hX = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in host_X]
+    hY = [torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory() for p in probs]
+
+    def one():
+        for i, p in enumerate(probs):
+            Xd = hX[i].to(device, non_blocking=True).view(torch.bfloat16)
+            xc, xs = w4.mxfp8_quant(Xd, w4.MX_SCALES_MMA)
+            hY[i].copy_(w4.mx_gemm(xc, xs, state[i][0], state[i][1], weights_static=True), non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    e1.synchronize()
+    barrier()
+    return {"ms": e0.elapsed_time(e1), "work": mx_step_bytes(probs) * steps,
+            "h2d": sum(x.numel() * 2 for x in hX), "d2h": sum(y.numel() * 2 for y in hY), "steps": steps,
+            "what": "H2D of X, w4_mxfp8_quant, w4_mx_gemm, D2H of Y (MXFP4 weights resident)"}
+
+
+def oracle_mx_prepare(oracle, probs, host_W, rows: int, offset: int = 0):
+    """Rows [offset, offset + rows) of each weight quantized to MXFP4 by the
+    oracle (model state, untimed)."""
+    out = []
+    for p, W in zip(probs, host_W):
+        r0 = offset % p.N
+        r1 = min(p.N, r0 + rows)
+        out.append(oracle.fp4_quant(np.ascontiguousarray(W[r0:r1]), MXFP4_KIND))
+    return out
+
+
+def oracle_mx_sample(oracle, probs, host_X, prepared) -> int:
+    """The oracle's share of one step: each layer's activations quantized to
+    MXFP8 and their fp64 product with the prepared weight rows.  Returns the
+    algorithmic bytes processed."""
+    nb = 0
+    for p, X, (wc, ws) in zip(probs, host_X, prepared):
+        xc, xs = oracle.mxfp8_quant(X)
+        oracle.mx_reference(xc, xs, wc, ws)
+        nb += roofline.mxfp8_quant_bytes(p.M, p.K) + roofline.mx_gemm_bytes(p.M, wc.shape[0], p.K)
+    return nb
+
+
+def cpu_baseline_mx(probs, host_W, host_X, budget_s):
+    import oracle
+    oracle.build()
+    rows = 16
+    prep = oracle_mx_prepare(oracle, probs, host_W, rows)
+    t0 = time.perf_counter()
+    oracle_mx_sample(oracle, probs, host_X, prep)
+    dt = time.perf_counter() - t0
+    rows = min(max(p.N for p in probs), max(16, int(16 * budget_s / max(dt, 1e-3))))
+    prep = oracle_mx_prepare(oracle, probs, host_W, rows)
+    t0 = time.perf_counter()
+    nb = oracle_mx_sample(oracle, probs, host_X, prep)
+    dt = time.perf_counter() - t0
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle", "seconds": round(dt, 2),
+            "sample": "first %d rows of each decode weight: oracle MXFP8 quantization of X and the fp64 product "
+                      "with those rows of the MXFP4 weight (quantized by the oracle beforehand, untimed), "
+                      "single thread" % rows}
+
+
+def run_reference_mx(args, world):
+    """The oracle on `rows` rows of each layer's weight per step (rotating)."""
+    import oracle
+    probs = synth.workload(args.workload)
+    host_W = [p.W() for p in probs]
+    host_X = [p.X() for p in probs]
+    rows = 16
+    steps_total = max(3, args.warmup) + args.steps
+    prep = {si: oracle_mx_prepare(oracle, probs, host_W, rows, si * rows) for si in range(steps_total)}
+    for si in range(max(3, args.warmup)):
+        oracle_mx_sample(oracle, probs, host_X, prep[si])
+    nb = 0
+    t0 = time.perf_counter()
+    for j in range(args.steps):
+        nb += oracle_mx_sample(oracle, probs, host_X, prep[max(3, args.warmup) + j])
+    dt = time.perf_counter() - t0
+    sample = ("%d rows of each weight per step (rotating): oracle MXFP8 quantization of X and the fp64 product "
+              "(weights quantized by the oracle before timing), single thread" % rows)
+    print_reference(args, world, nb / dt / 1e9, "GB/s", dt * 1e3 / args.steps, WORKLOAD_DESC[args.workload], sample)
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
@@ -1128,6 +1430,9 @@ def main(argv=None):
         return 0
     if args.workload == "fp4quant":
         run_fp4(args, rank, world, local_rank)
+        return 0
+    if args.workload in MX_WORKLOADS:
+        run_mx(args, rank, world, local_rank)
         return 0
     run_w4(args, rank, world, local_rank)
     return 0

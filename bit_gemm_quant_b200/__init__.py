@@ -58,9 +58,7 @@ def lib() -> ctypes.CDLL:
         L.w4_mxfp8_quant.restype = I
         L.w4_mx_scale_layout.argtypes = [P, I64, I64, P, P]
         L.w4_mx_scale_layout.restype = I
-        L.w4_mx_workspace_bytes.argtypes = [I64, I64, I64]
-        L.w4_mx_workspace_bytes.restype = SZ
-        L.w4_mx_gemm.argtypes = [P, P, I64, I64, I64, P, P, P, P, SZ, P]
+        L.w4_mx_gemm.argtypes = [P, P, I64, I64, I64, P, P, P, I, P]
         L.w4_mx_gemm.restype = I
         L.w4_status_string.argtypes = [I]
         L.w4_status_string.restype = ctypes.c_char_p
@@ -117,12 +115,8 @@ def w4_mx_scale_layout(src, R, K, dst, stream) -> int:
     return lib().w4_mx_scale_layout(src, R, K, dst, stream)
 
 
-def w4_mx_workspace_bytes(M, N, K) -> int:
-    return int(lib().w4_mx_workspace_bytes(M, N, K))
-
-
-def w4_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, workspace, workspace_bytes, stream) -> int:
-    return lib().w4_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, workspace, workspace_bytes, stream)
+def w4_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, flags, stream) -> int:
+    return lib().w4_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, flags, stream)
 
 
 def w4_status_string(status: int) -> str:
@@ -297,19 +291,16 @@ def mx_scale_layout(scales_rows, K: int, stream=None, out=None):
     return dst
 
 
-def mx_gemm(x_codes, x_scales, w_codes, w_scales, workspace=None, out=None, stream=None):
+def mx_gemm(x_codes, x_scales, w_codes, w_scales, out=None, stream=None, weights_static: bool = False):
     """Y[M,N] bf16 = X^ . W^^T from MXFP8 activations (codes [M,K], tensor-core
-    layout scales) and MXFP4 weights (codes [N,K/2], tensor-core layout scales)."""
+    layout scales) and MXFP4 weights (codes [N,K/2], tensor-core layout scales).
+    ``weights_static`` passes W4_WEIGHTS_STATIC (see ``gemm``)."""
     import torch
     M, K = x_codes.shape
     N = w_codes.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device)
-    need = w4_mx_workspace_bytes(M, N, K)
-    if need and workspace is None:
-        workspace = torch.zeros(need, dtype=torch.uint8, device=x_codes.device)
-    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = w4_mx_gemm(_ptr(x_codes), _ptr(x_scales), M, N, K, _ptr(w_codes), _ptr(w_scales), _ptr(Y), _ptr(workspace),
-                    wbytes, _stream_handle(stream))
+    st = w4_mx_gemm(_ptr(x_codes), _ptr(x_scales), M, N, K, _ptr(w_codes), _ptr(w_scales), _ptr(Y),
+                    WEIGHTS_STATIC if weights_static else 0, _stream_handle(stream))
     if st != W4_OK:
         raise W4Error(st, "w4_mx_gemm")
     return Y

@@ -118,26 +118,18 @@ bool mx_shape_supported(int64_t M, int64_t N, int64_t K)
 }
 }  // namespace
 
-size_t w4_mx_workspace_bytes(int64_t M, int64_t N, int64_t K)
-{
-    if (!mx_shape_ok(M, N, K) || !mx_shape_supported(M, N, K)) return 0;
-    return w4::mx_workspace_bytes(M, N, K);
-}
-
 w4_status w4_mx_gemm(const uint8_t *x_codes, const uint8_t *x_scales, int64_t M, int64_t N, int64_t K,
-                     const uint8_t *w_codes, const uint8_t *w_scales, void *Y, void *workspace,
-                     size_t workspace_bytes, w4_stream_t stream)
+                     const uint8_t *w_codes, const uint8_t *w_scales, void *Y, int flags, w4_stream_t stream)
 {
     if (!x_codes || !x_scales || !w_codes || !w_scales || !Y) return W4_ERR_INVALID_ARG;
+    if ((flags & ~W4_WEIGHTS_STATIC) != 0) return W4_ERR_INVALID_ARG;
     if (!mx_shape_ok(M, N, K)) return W4_ERR_INVALID_ARG;
     if (!aligned(x_codes, 16) || !aligned(x_scales, 16) || !aligned(w_codes, 32) || !aligned(w_scales, 16) ||
         !aligned(Y, 2))
         return W4_ERR_INVALID_ARG;
     if (!mx_shape_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
-    const size_t need = w4::mx_workspace_bytes(M, N, K);
-    if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256)))) return W4_ERR_INVALID_ARG;
-    const cudaError_t e =
-        w4::launch_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y, workspace, (cudaStream_t)stream);
+    const cudaError_t e = w4::launch_mx_gemm(x_codes, x_scales, M, N, K, w_codes, w_scales, Y,
+                                             (flags & W4_WEIGHTS_STATIC) != 0, (cudaStream_t)stream);
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 

@@ -95,9 +95,9 @@ int64_t mx_padded_rows(int64_t R);
 cudaError_t launch_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales, int layout,
                                cudaStream_t stream);
 cudaError_t launch_mx_scale_layout(const uint8_t *src, int64_t R, int64_t K, uint8_t *dst, cudaStream_t stream);
-size_t mx_workspace_bytes(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_mx_gemm(const uint8_t *x_codes, const uint8_t *x_sf, int64_t M, int64_t N, int64_t K,
-                           const uint8_t *w_codes, const uint8_t *w_sf, void *Y, void *ws, cudaStream_t stream);
+                           const uint8_t *w_codes, const uint8_t *w_sf, void *Y, bool weights_static,
+                           cudaStream_t stream);
 size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
 // byte range of the split-K tile counters inside that workspace (0 bytes if none)
 void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size_t *bytes);

@@ -36,12 +36,20 @@
 // the copy for one stage never overwrites scales an MMA may still read.
 //
 // Split-K: when the tile grid leaves SMs idle, the 128-wide k-stages are split
-// across CTAs so that every CTA of the grid is resident at once; each writes
-// an fp32 partial tile to the caller's workspace and the last CTA of a tile
-// (an atomic counter) sums the partials in split order, writes Y and re-zeroes
-// the counter.  Every wait is bounded in time; a wait that runs out records an
-// error code (read by w4_device_error), raises a CTA-wide abort flag, and the
-// CTA drains its own copies and MMAs, frees its tensor memory and returns.
+// across the CTAs of a thread-block cluster (at most 8), sized so that every
+// CTA of the grid is resident at once.  Each CTA parks its fp32 partial tile in
+// its own (by then idle) shared memory; after a cluster barrier the first CTA
+// of the cluster reads the others' partials through distributed shared memory,
+// sums them in split order (the result does not depend on timing) and writes
+// Y; a second cluster barrier keeps every partial alive until it has been read.
+// With W4_WEIGHTS_STATIC the weight copies of the first ring of stages are
+// issued before the kernel waits for the previous one on the stream; the
+// activations wait.  (An L2 prefetch of the rest of each CTA's weight slice at
+// that point made the kernel slower and is not done.)
+// Every wait on a copy or an MMA is bounded in time; a wait that runs out
+// records an error code (read by w4_device_error), raises a CTA-wide abort
+// flag, and the CTA drains its own copies and MMAs, takes part in the cluster
+// barriers, frees its tensor memory and returns.
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -115,6 +123,33 @@ __device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// The shared::cluster address of `addr` (a shared::cta address) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_cluster(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 __device__ __noinline__ bool mx_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *err, int code,
                                      uint64_t limit)
 {
@@ -143,12 +178,11 @@ __device__ __noinline__ void mx_drain(uint64_t *bar, uint32_t parity, int *err)
     }
 }
 
-template <int BN>
+template <int BN, bool EARLY>
 __global__ void __launch_bounds__(kMxThreads, MxCfg<BN>::kPerSM)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                const uint8_t *__restrict__ w_sf, const uint8_t *__restrict__ x_sf, int M, int N, int K,
-               __nv_bfloat16 *__restrict__ Y, float *__restrict__ partial, unsigned *__restrict__ counters,
-               int splits, int ks_per_split, int *err, uint64_t wait_ns)
+               __nv_bfloat16 *__restrict__ Y, int splits, int ks_per_split, int *err, uint64_t wait_ns)
 {
     using C = MxCfg<BN>;
     constexpr int S = C::kStages;
@@ -160,7 +194,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     uint64_t *stall = done + 1;                       // a barrier nothing completes (failure tests)
     uint32_t *tmem_slot = (uint32_t *)(stall + 1);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-    int *last_flag = (int *)(tmem_slot + 2);
     const uint64_t limit = wait_limit_of(wait_ns);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,7 +216,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         mbar_init(done, 1);
         mbar_init(stall, 1);
         *abort_flag = 0;
-        *last_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::kCols);
@@ -191,30 +223,52 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
+
+    const uint32_t tx = 128 * kMxKS / 2 + C::kBBytes + 512 + 512 * nsfb;
+    const uint8_t *sfa_src = w_sf + ((size_t)(n0 >> 7) * KS + ks_begin) * 512;
+    const uint8_t *sfb_src = x_sf + ((size_t)(m0 >> 7) * KS + ks_begin) * 512;
+    const int first = min(nks, S);               // stages whose ring slots are free at the start
+    auto issue_w = [&](int i) {                  // weight half of stage i (codes + scale atom)
+        const int s = i % S;
+        uint8_t *st = smem + s * C::kStageBytes;
+        tma_load_2d(st, &tmap_w, &full[s], (ks_begin + i) * kMxKS, n0);
+        bulk_load(st + C::kSfaOff, sfa_src + (size_t)i * 512, 512, &full[s]);
+    };
+    auto issue_x = [&](int i) {                  // activation half of stage i
+        const int s = i % S;
+        uint8_t *st = smem + s * C::kStageBytes;
+        tma_load_2d(st + C::kABytes, &tmap_x, &full[s], (ks_begin + i) * kMxKS, m0);
+        for (int j = 0; j < nsfb; ++j)
+            bulk_load(st + C::kSfbOff + 512 * j, sfb_src + ((size_t)j * KS + i) * 512, 512, &full[s]);
+    };
+    if (EARLY && warp == 0 && lane == 0) {
+        // the weights are not written by the previous kernel: start streaming them now
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_w) : "memory");
+        for (int i = 0; i < first; ++i) {
+            mbar_arrive_expect_tx(&full[i], tx);
+            issue_w(i);
+        }
+    }
+    pdl_wait();                                   // the activations (and, without EARLY, everything) are ready
     pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ copy producer --
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_w) : "memory");
+            if (!EARLY) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_w) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(&tmap_x) : "memory");
-            const uint32_t tx = 128 * kMxKS / 2 + C::kBBytes + 512 + 512 * nsfb;
-            const uint8_t *sfa_src = w_sf + ((size_t)(n0 >> 7) * KS + ks_begin) * 512;
-            const uint8_t *sfb_src = x_sf + ((size_t)(m0 >> 7) * KS + ks_begin) * 512;
             int issued = 0;
-            for (int i = 0; i < nks; ++i) {
+            if (EARLY) {
+                for (int i = 0; i < first; ++i) issue_x(i);
+                issued = first;
+            }
+            for (int i = issued; i < nks; ++i) {
                 const int s = i % S;
                 const uint32_t ph = (i / S) & 1;
                 if (!mx_wait(&empty[s], ph ^ 1, abort_flag, err, kErrMxWaitEmpty, limit)) break;
-                uint8_t *st = smem + s * C::kStageBytes;
-                const int k = (ks_begin + i) * kMxKS;
                 mbar_arrive_expect_tx(&full[s], tx);
-                tma_load_2d(st, &tmap_w, &full[s], k, n0);
-                tma_load_2d(st + C::kABytes, &tmap_x, &full[s], k, m0);
-                bulk_load(st + C::kSfaOff, sfa_src + (size_t)i * 512, 512, &full[s]);
-                for (int j = 0; j < nsfb; ++j)
-                    bulk_load(st + C::kSfbOff + 512 * j, sfb_src + ((size_t)j * KS + i) * 512, 512, &full[s]);
+                issue_w(i);
+                issue_x(i);
                 ++issued;
             }
             // every issued copy must have landed before the CTA may exit
@@ -260,9 +314,12 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const bool have =
             __all_sync(0xffffffffu, mx_wait(done, 0, abort_flag, err, kErrMxWaitDone, limit) && *abort_flag == 0);
         tc_fence_after();
+        // columns (tokens) of this tile that exist
+        const int cols = min(BN, M - m0);
+        float *red = (float *)smem;                  // [BN][128] fp32 partial, in the idle ring
         if (have) {
             constexpr int CH = BN < 32 ? BN : 32;
-            for (int c = 0; c < BN; c += CH) {
+            for (int c = 0; c < cols; c += CH) {
                 float acc[CH];
                 if constexpr (CH == 32) {
                     tmem_ld32(lane_addr + c, acc);
@@ -273,38 +330,45 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < CH; ++j) {
-                    const int m = m0 + c + j;
-                    if (okn && m < M) {
-                        if (splits == 1) Y[(size_t)m * N + n] = __float2bfloat16_rn(acc[j]);
-                        else partial[((size_t)split * M + m) * N + n] = acc[j];
+                    if (c + j < cols) {
+                        if (splits == 1) {
+                            if (okn) Y[(size_t)(m0 + c + j) * N + n] = __float2bfloat16_rn(acc[j]);
+                        } else {
+                            red[(c + j) * 128 + 32 * q + lane] = acc[j];
+                        }
                     }
                 }
             }
         }
-        if (splits > 1) {
-            // the counter protocol runs even after an abort, so that the tile's
-            // counter is re-zeroed (Y is then undefined and the error recorded)
-            __threadfence();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (threadIdx.x == 64) {
-                const unsigned tile = blockIdx.y * gridDim.x + blockIdx.x;
-                const unsigned prev = atomicAdd(&counters[tile], 1u);
-                *last_flag = (prev == (unsigned)splits - 1) ? 1 : 0;
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (*(volatile int *)last_flag) {
-                __threadfence();
-                for (int c = 0; c < BN; ++c) {
-                    const int m = m0 + c;
-                    if (okn && m < M) {
-                        float sum = 0.f;
-                        for (int sp = 0; sp < splits; ++sp) sum += __ldcg(partial + ((size_t)sp * M + m) * N + n);
-                        Y[(size_t)m * N + n] = __float2bfloat16_rn(sum);
-                    }
+    }
+
+    if (splits > 1) {
+        // split-K across the cluster: partials are summed in split order by the
+        // cluster's first CTA (every thread of every CTA takes part in both
+        // barriers, also after an abort, when Y is left undefined)
+        cluster_sync_all();
+        if (cluster_rank() == 0 && warp >= 2) {
+            const int q = warp & 3;
+            const int r = 32 * q + lane;
+            const int n = n0 + r;
+            const int cols = min(BN, M - m0);
+            const uint32_t red0 = smem_u32(smem);
+            if (n < N) {
+                for (int c = 0; c < cols; ++c) {
+                    const uint32_t a = red0 + (uint32_t)((c * 128 + r) * 4);
+                    float v[8];
+#pragma unroll
+                    for (int sp = 0; sp < 8; ++sp)
+                        if (sp < splits) v[sp] = ld_cluster_f32(map_cluster(a, (uint32_t)sp));
+                    float sum = v[0];
+#pragma unroll
+                    for (int sp = 1; sp < 8; ++sp)
+                        if (sp < splits) sum += v[sp];
+                    Y[(size_t)(m0 + c) * N + n] = __float2bfloat16_rn(sum);
                 }
-                if (threadIdx.x == 64) counters[blockIdx.y * gridDim.x + blockIdx.x] = 0u;
             }
         }
+        cluster_sync_all();
     }
 
     tc_fence_before();
@@ -317,8 +381,9 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 
 struct MxPlan {
     int BN = 0, m_tiles = 0, n_tiles = 0, splits = 1, ks_per_split = 0;
-    size_t ws_bytes = 0;
 };
+
+constexpr int kMxMaxSplits = 8;                 // portable cluster size
 
 int mx_pick_bn(int64_t M)
 {
@@ -338,55 +403,71 @@ MxPlan plan_mx(int64_t M, int64_t N, int64_t K)
     const int KS = (int)(K / kMxKS);
     const int64_t tiles = (int64_t)p.m_tiles * p.n_tiles;
     const int64_t slots = (int64_t)kNumSMs * (p.BN <= 64 ? 2 : 1);
-    // the most splits (at least two k-stages each) whose grid is resident at
-    // once: HBM is then shared by every CTA of the grid and none waits for a
-    // second wave
+    // the most splits (at least two k-stages each, at most one cluster) whose
+    // grid is resident at once: HBM is then shared by every CTA of the grid and
+    // none waits for a second wave.  Clusters are placed within GPCs, which
+    // strands some CTA slots: a grid of 96 three-CTA clusters (288 CTAs of 296
+    // slots) ran partly in a second wave, 86 of them (258 CTAs) did not, so
+    // split grids keep 10% of the slots free.
+    const int64_t cluster_slots = slots * 9 / 10;
     int per = KS;
-    for (int s = 2; s <= KS / 2; ++s) {
+    for (int s = 2; s <= KS / 2 && s <= kMxMaxSplits; ++s) {
         const int per_s = (KS + s - 1) / s;
         const int s_eff = (KS + per_s - 1) / per_s;
-        if (tiles * s_eff > slots) break;
+        if (tiles * s_eff > cluster_slots) break;
         per = per_s;
     }
     p.ks_per_split = per;
     p.splits = (KS + per - 1) / per;
-    if (p.splits > 1) {
-        const size_t part = (size_t)p.splits * M * N * sizeof(float);
-        p.ws_bytes = ((part + 255) & ~(size_t)255) + (size_t)tiles * sizeof(unsigned);
-    }
     return p;
 }
 
-template <int BN>
+template <int BN, bool EARLY>
 cudaError_t mx_launch_bn(const CUtensorMap &wmap, const CUtensorMap &xmap, const MxPlan &p, int M, int N, int K,
-                         const uint8_t *w_sf, const uint8_t *x_sf, void *Y, void *ws, cudaStream_t stream)
+                         const uint8_t *w_codes, const uint8_t *w_sf, const uint8_t *x_sf, void *Y,
+                         cudaStream_t stream)
 {
     using C = MxCfg<BN>;
+    auto kern = mx_gemm_kernel<BN, EARLY>;
     static std::atomic<bool> attr_done[kMaxDevices];
     {
-        const cudaError_t e = set_smem_attr(mx_gemm_kernel<BN>, C::kSmem, attr_done);
+        const cudaError_t e = set_smem_attr(kern, C::kSmem, attr_done);
         if (e != cudaSuccess) return e;
-    }
-    float *partial = nullptr;
-    unsigned *counters = nullptr;
-    if (p.splits > 1) {
-        const size_t part = (size_t)p.splits * M * N * sizeof(float);
-        partial = (float *)ws;
-        counters = (unsigned *)((uint8_t *)ws + ((part + 255) & ~(size_t)255));
     }
     int *err = device_error_word();
     if (!err) return cudaErrorUnknown;
-    dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    return launch_pdl(mx_gemm_kernel<BN>, grid, dim3(kMxThreads), C::kSmem, stream, wmap, xmap, w_sf, x_sf, M, N, K,
-                      (__nv_bfloat16 *)Y, partial, counters, p.splits, p.ks_per_split, err, wait_limit_ns());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_tiles, p.m_tiles, p.splits);
+    cfg.blockDim = dim3(kMxThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = (unsigned)p.splits;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.splits > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kern, wmap, xmap, w_sf, x_sf, M, N, K, (__nv_bfloat16 *)Y, p.splits,
+                              p.ks_per_split, err, wait_limit_ns());
+}
+
+template <int BN>
+cudaError_t mx_launch_early(bool early, const CUtensorMap &wmap, const CUtensorMap &xmap, const MxPlan &p, int M,
+                            int N, int K, const uint8_t *w_codes, const uint8_t *w_sf, const uint8_t *x_sf, void *Y,
+                            cudaStream_t stream)
+{
+    if (early) return mx_launch_bn<BN, true>(wmap, xmap, p, M, N, K, w_codes, w_sf, x_sf, Y, stream);
+    return mx_launch_bn<BN, false>(wmap, xmap, p, M, N, K, w_codes, w_sf, x_sf, Y, stream);
 }
 
 }  // namespace
 
-size_t mx_workspace_bytes(int64_t M, int64_t N, int64_t K) { return plan_mx(M, N, K).ws_bytes; }
-
 cudaError_t launch_mx_gemm(const uint8_t *x_codes, const uint8_t *x_sf, int64_t M, int64_t N, int64_t K,
-                           const uint8_t *w_codes, const uint8_t *w_sf, void *Y, void *ws, cudaStream_t stream)
+                           const uint8_t *w_codes, const uint8_t *w_sf, void *Y, bool weights_static,
+                           cudaStream_t stream)
 {
     const MxPlan p = plan_mx(M, N, K);
     EncodeTiledFn enc = encode_fn();
@@ -411,12 +492,13 @@ cudaError_t launch_mx_gemm(const uint8_t *x_codes, const uint8_t *x_sf, int64_t 
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    const bool e = weights_static;
     switch (p.BN) {
-    case 16: return mx_launch_bn<16>(wmap, xmap, p, (int)M, (int)N, (int)K, w_sf, x_sf, Y, ws, stream);
-    case 32: return mx_launch_bn<32>(wmap, xmap, p, (int)M, (int)N, (int)K, w_sf, x_sf, Y, ws, stream);
-    case 64: return mx_launch_bn<64>(wmap, xmap, p, (int)M, (int)N, (int)K, w_sf, x_sf, Y, ws, stream);
-    case 128: return mx_launch_bn<128>(wmap, xmap, p, (int)M, (int)N, (int)K, w_sf, x_sf, Y, ws, stream);
-    default: return mx_launch_bn<256>(wmap, xmap, p, (int)M, (int)N, (int)K, w_sf, x_sf, Y, ws, stream);
+    case 16: return mx_launch_early<16>(e, wmap, xmap, p, (int)M, (int)N, (int)K, w_codes, w_sf, x_sf, Y, stream);
+    case 32: return mx_launch_early<32>(e, wmap, xmap, p, (int)M, (int)N, (int)K, w_codes, w_sf, x_sf, Y, stream);
+    case 64: return mx_launch_early<64>(e, wmap, xmap, p, (int)M, (int)N, (int)K, w_codes, w_sf, x_sf, Y, stream);
+    case 128: return mx_launch_early<128>(e, wmap, xmap, p, (int)M, (int)N, (int)K, w_codes, w_sf, x_sf, Y, stream);
+    default: return mx_launch_early<256>(e, wmap, xmap, p, (int)M, (int)N, (int)K, w_codes, w_sf, x_sf, Y, stream);
     }
 }
 

@@ -10,6 +10,10 @@ must read and write once (not DRAM counters):
   FLOPs of w4a16_gemm:     2 M N K
   w4_fp4_quant(N, K, B):   read W (2NK), write codes (NK/2) and one scale byte
                            per block of B (N K/B)
+  w4_mxfp8_quant(M, K):    read X (2MK), write codes (MK) and scales (MK/32)
+  w4_mx_gemm(M, N, K):     read weight codes (NK/2) and scales (NK/32),
+                           activation codes (MK) and scales (MK/32), write Y (2MN)
+  FLOPs of w4_mx_gemm:     2 M N K
 """
 from __future__ import annotations
 
@@ -37,6 +41,14 @@ def gemm_bytes(M: int, N: int, K: int, g: int, mode: int) -> int:
 
 def fp4_quant_bytes(N: int, K: int, block: int) -> int:
     return 2 * N * K + N * K // 2 + N * (K // block)
+
+
+def mxfp8_quant_bytes(M: int, K: int) -> int:
+    return 2 * M * K + M * K + M * K // 32
+
+
+def mx_gemm_bytes(M: int, N: int, K: int) -> int:
+    return N * K // 2 + N * K // 32 + M * K + M * K // 32 + 2 * M * N
 
 
 def gemm_flops(M: int, N: int, K: int) -> int:

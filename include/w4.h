@@ -80,7 +80,7 @@ typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
 
 /*
  * W4_WEIGHTS_STATIC -- a flag OR-ed into the `mode` argument of w4a16_gemm and
- * w4a16_gemm_noalloc (never of w4_quant_pack).  It declares that the packed
+ * w4a16_gemm_noalloc (never of w4_quant_pack), and the `flags` of w4_mx_gemm.  It declares that the packed
  * weight, its scales and its zero-points are NOT written by the kernel that
  * immediately precedes this call on `stream` -- the usual case for model
  * weights quantized once at load time.  The product may then start reading
@@ -290,37 +290,29 @@ w4_status w4_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, ui
 w4_status w4_mx_scale_layout(const uint8_t *src, int64_t R, int64_t K, uint8_t *dst, w4_stream_t stream);
 
 /*
- * w4_mx_workspace_bytes -- device scratch that w4_mx_gemm needs for this
- * shape (split-K partial sums and tile counters), 0 if none.  Same contract
- * as w4a16_workspace_bytes: zero-filled before its first use with a shape,
- * left zero-filled by every successful call.
- */
-size_t w4_mx_workspace_bytes(int64_t M, int64_t N, int64_t K);
-
-/*
  * w4_mx_gemm -- Y = X^ . W^^T for MXFP8 activations and MXFP4 weights on the
  * block-scaled tensor cores (page 3 section 4.3: FP4 weights times FP8
  * activations, E8M0 scales per 32; page 2, the Blackwell FP4 paragraph: the
  * block-scaled format feeds the tensor cores directly).
  *   Y[m][n] = bf16_rne(sum_k x^[m][k] * w^[n][k]) with x^ from
  *   w4_mxfp8_quant, w^ from w4_fp4_quant(W4_MXFP4) (w^ = e2m1(code) * 2^e),
- *   accumulated by the tensor cores in fp32 (the summation order is the
- *   hardware's).
+ *   accumulated by the tensor cores in fp32; a split of k across CTAs adds
+ *   its fp32 partial sums in a fixed order, so results repeat bit for bit.
  *   x_codes  uint8 [M][K] E4M3 codes, 16-byte aligned.
  *   x_scales E8M0, W4_MX_SCALES_MMA layout for M rows, 16-byte aligned.
  *   M, N, K  M >= 1, N >= 1, K >= 128, K % 128 == 0.
  *   w_codes  uint8 [N][K/2] MXFP4 codes (w4_fp4_quant layout), 32-byte aligned.
  *   w_scales E8M0, W4_MX_SCALES_MMA layout for N rows, 16-byte aligned.
  *   Y        out, bf16 [M][N], 2-byte aligned.
- *   workspace, workspace_bytes: w4_mx_workspace_bytes(M, N, K) bytes,
- *            256-byte aligned (may be NULL when that is 0).
- * Errors: W4_ERR_INVALID_ARG for a NULL or misaligned pointer, a bad size or
- * a short workspace; W4_ERR_UNSUPPORTED for shapes past 32-bit indexing;
- * W4_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ *   flags    0 or W4_WEIGHTS_STATIC (as for w4a16_gemm: the weight codes and
+ *            scales are not written by the kernel right before this call on
+ *            `stream`, so their stream may start before it finishes).
+ * Needs no workspace.  Errors: W4_ERR_INVALID_ARG for a NULL or misaligned
+ * pointer, a bad size or flag; W4_ERR_UNSUPPORTED for shapes past 32-bit
+ * indexing; W4_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
  */
 w4_status w4_mx_gemm(const uint8_t *x_codes, const uint8_t *x_scales, int64_t M, int64_t N, int64_t K,
-                     const uint8_t *w_codes, const uint8_t *w_scales, void *Y, void *workspace,
-                     size_t workspace_bytes, w4_stream_t stream);
+                     const uint8_t *w_codes, const uint8_t *w_scales, void *Y, int flags, w4_stream_t stream);
 
 /* Text for a status code; never NULL. */
 const char *w4_status_string(int status);

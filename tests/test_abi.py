@@ -225,9 +225,9 @@ def test_mx_scale_layout_rejects_bad_arguments(w4):
     assert f(src=FAKE + 2) == E and f(dst=FAKE + 8) == E
 
 
-def mxg(w4, xc=FAKE, xs=FAKE, M=1, N=256, K=512, wc=FAKE, wsf=FAKE, Y=FAKE, ws=None, wsb=0):
+def mxg(w4, xc=FAKE, xs=FAKE, M=1, N=256, K=512, wc=FAKE, wsf=FAKE, Y=FAKE, flags=0):
     return w4.w4_mx_gemm(P(xc) if xc else None, P(xs) if xs else None, M, N, K, P(wc) if wc else None,
-                         P(wsf) if wsf else None, P(Y) if Y else None, P(ws) if ws else None, wsb, None)
+                         P(wsf) if wsf else None, P(Y) if Y else None, flags, None)
 
 
 def test_mx_gemm_rejects_bad_arguments(w4):
@@ -239,16 +239,5 @@ def test_mx_gemm_rejects_bad_arguments(w4):
     assert mxg(w4, wc=FAKE + 16) == E                         # the FP4 tensor map wants 32-byte alignment
     assert mxg(w4, xc=FAKE + 8) == E and mxg(w4, xs=FAKE + 8) == E and mxg(w4, wsf=FAKE + 4) == E
     assert mxg(w4, Y=FAKE + 1) == E
-    # a shape that splits k needs its workspace
-    need = w4.w4_mx_workspace_bytes(1, 4096, 4096)
-    assert need > 0
-    assert mxg(w4, N=4096, K=4096) == E
-    assert mxg(w4, N=4096, K=4096, ws=FAKE, wsb=need - 1) == E
-    assert mxg(w4, N=4096, K=4096, ws=FAKE + 64, wsb=need) == E
-
-
-def test_mx_workspace_query_is_host_only(w4):
-    assert w4.w4_mx_workspace_bytes(1, 4096, 4096) > 0        # 32 tiles: k is split
-    assert w4.w4_mx_workspace_bytes(1, 28672, 8192) == 0      # 224 tiles fill the SMs
-    assert w4.w4_mx_workspace_bytes(1, 4096, 4000) == 0       # malformed
-    assert w4.w4_mx_workspace_bytes(0, 4096, 4096) == 0
+    assert mxg(w4, flags=1) == E and mxg(w4, flags=0x300) == E   # W4_WEIGHTS_STATIC is the only flag
+    assert mxg(w4, M=1 << 40, K=1 << 30) == E                 # M*K overflows int64

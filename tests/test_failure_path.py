@@ -83,3 +83,26 @@ def test_quantizer_wait_runs_out_then_next_call_is_correct(w4):
     oq, osc, _ = oracle.quant_pack(W, 128, SYM, threads=THREADS)
     assert_codes_equal(host_u32(q), oq, "qweight")
     assert_codes_equal(host_u16(sc), osc, "scales")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (200, 512, 1024)], ids=["split_cluster", "single"])
+def test_mx_product_wait_runs_out_then_next_call_is_correct(w4, M, N, K):
+    """The block-scaled product: the MMA issuer's first wait runs out; the CTA
+    drains its copies, still takes part in the cluster barriers of a split-k
+    grid, frees its tensor memory and the next call is correct."""
+    import torch
+    from test_parity_mx import oracle_chain
+    from parity import assert_y_elementwise
+    W = synth.weights(81, N, K, 0.02, 0.01, 5.0)
+    X = synth.activations(82, M, K, 0.01, 40.0)
+    wc, ws_rows = w4.fp4_quant(dev_bf16(W), w4.MXFP4)
+    ws = w4.mx_scale_layout(ws_rows, K)
+    xc, xs = w4.mxfp8_quant(dev_bf16(X), w4.MX_SCALES_MMA)
+    code = run_with_short_limit(w4, lambda: w4.mx_gemm(xc, xs, wc, ws))
+    assert 0x301 <= code <= 0x304, hex(code)
+    Y = host_bf16_as_f64(w4.mx_gemm(xc, xs, wc, ws))
+    torch.cuda.synchronize()
+    assert w4.w4_device_error() == 0
+    Y_ref, Y_abs = oracle_chain(X, W)[:2]
+    assert_y_elementwise(Y, Y_ref, Y_abs, K, "Y after a failed call")

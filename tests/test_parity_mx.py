@@ -167,13 +167,15 @@ def test_mx_gemm_matches_the_oracle(w4, M, N, K):
 @pytest.mark.gpu
 def test_mx_gemm_repeats_bit_for_bit(w4):
     """Split-K partials are summed in split order: the result does not depend
-    on which CTA finishes last."""
+    on which CTA finishes first; W4_WEIGHTS_STATIC gives the same bits."""
     import torch
     W = synth.weights(23, 4096, 4096, std=0.02)
     X = synth.activations(24, 1, 4096)
-    Y0 = gpu_chain(w4, X, W)[0]
-    for _ in range(3):
-        assert torch.equal(gpu_chain(w4, X, W)[0], Y0)
+    Y0, wc, _, _ = gpu_chain(w4, X, W)
+    ws = w4.mx_scale_layout(w4.fp4_quant(dev_bf16(W), w4.MXFP4)[1], 4096)
+    xc, xs = w4.mxfp8_quant(dev_bf16(X), w4.MX_SCALES_MMA)
+    for static in (False, True, False, True):
+        assert torch.equal(w4.mx_gemm(xc, xs, wc, ws, weights_static=static), Y0)
 
 
 @pytest.mark.gpu
