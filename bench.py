@@ -35,7 +35,10 @@ inside the step graph would cost several microseconds per kernel.)
 
 Under torchrun (N > 1) every rank runs its own replica with its own seeds
 (weak scaling, no collective on the data path); the timed region is bracketed
-by barriers and the reported time is the max over ranks.  Rank 0 prints one
+by barriers and the reported time is the max over ranks.  With --shard n|k the
+product workloads scale strongly instead: every layer is split over the ranks
+(bit_gemm_quant_b200.shard), and a step includes the collective that
+completes Y.  Rank 0 prints one
 JSON line.  ``--impl reference`` times the CPU oracle on a bounded sample of
 the same workload instead (rank 0 only).
 """
@@ -75,6 +78,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", choices=["decode", "smallbatch", "prefill", "quantizer", "decodequant", "awq", "fp4quant",
                                                "mxdecode"],
                     default="decode")
+    ap.add_argument("--shard", choices=["none", "n", "k"], default="none",
+                    help="strong scaling of the product workloads: split every layer over the ranks by rows of W "
+                         "(n, all-gather of Y) or by columns (k, all-reduce of fp32 partials); default: replicas")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1419,6 +1425,156 @@ def run_reference_mx(args, world):
     print_reference(args, world, nb / dt / 1e9, "GB/s", dt * 1e3 / args.steps, WORKLOAD_DESC[args.workload], sample)
 
 
+# ------------------------------------------------ strong scaling (sharded) --
+
+def run_sharded(args, rank, world, local_rank):
+    """Every layer of a product workload split over the ranks: rows of W
+    (column-parallel, all-gather of Y) or columns of W and X (row-parallel,
+    all-reduce of the fp32 partials, then the bf16 rounding).  All ranks hold
+    shares of the same layers (same seeds); value = the unsharded layers'
+    algorithmic bytes (FLOPs for prefill) per step / the max-over-ranks time."""
+    import torch
+    import bit_gemm_quant_b200 as w4
+    from bit_gemm_quant_b200 import shard
+
+    if args.workload not in ("decode", "smallbatch", "prefill"):
+        raise SystemExit("--shard applies to the product workloads (decode, smallbatch, prefill)")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    pg_ok = world > 1
+    if pg_ok:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+    w4.lib()
+    pk = roofline.peaks(ROOT)
+    split = args.shard
+    plist = problems_for(args.workload)
+    keys = list(dict.fromkeys(k for k, _ in plist))
+    first = {k: p for k, p in reversed(plist)}
+    qp = {k: first[k] for k in keys}
+    dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+    layers = {}
+    for k in keys:
+        p = qp[k]
+        W = synth.weights(p.seed, p.N, p.K, p.w_std, *p.w_outlier)
+        layers[k] = shard.ShardedW4Linear(dev(shard.local_weight(W, split, world, rank, p.group)), p.N, p.K, p.group,
+                                          p.mode, split, world, rank)
+    host_X = {p.name: shard.local_activations(p.X(), split, world, rank, p.group) for _, p in plist}
+    X_d = {n: dev(x) for n, x in host_X.items()}
+    torch.cuda.synchronize()
+
+    def step():
+        for key, p in plist:
+            layers[key].forward(X_d[p.name])
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(smi_gpu_id(local_rank))
+    sampler.start()
+    sampler.mark_begin()
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        step()
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    e1.synchronize()
+    barrier()
+    local_ms = e0.elapsed_time(e1)
+    sampler.mark_end()
+    clocks = sampler.stop()
+
+    prefill = args.workload == "prefill"
+    per_step = sum((roofline.gemm_flops(p.M, p.N, p.K) if prefill else roofline.gemm_bytes(p.M, p.N, p.K, p.group, p.mode))
+                   for _, p in plist)
+    # strong scaling: the work is the unsharded layers', counted once (not per rank)
+    max_ms, _ = aggregate(local_ms, 0.0, device)
+    value = args.steps * per_step / (max_ms * 1e-3) / (1e12 if prefill else 1e9)
+
+    # the local product alone (no collective): its algorithmic bytes over its time
+    KL = max(args.steps, 50)
+    loc = []
+    for key, p in plist:
+        lay = layers[key]
+        n_loc, k_loc = lay.n1 - lay.n0, lay.k1 - lay.k0
+        f = (lambda lay=lay, x=X_d[p.name], n=n_loc: lay.ops.gemm(x, lay.packed, lay.group, lay.mode,
+                                                                   n, out_f32=lay.split == "k"))
+        avg, _ = graph_launch_ms(torch, device, [f], KL)
+        loc.append((roofline.gemm_bytes(p.M, n_loc, k_loc, p.group, p.mode), roofline.gemm_flops(p.M, n_loc, k_loc),
+                    avg))
+    nb = sum(b for b, _, _ in loc) / len(loc)
+    nf = sum(f for _, f, _ in loc) / len(loc)
+    avg_ms = sum(t for _, _, t in loc) / len(loc)
+    if prefill:
+        ach = nf / (avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(ach / pk["bf16_tflops"], 4)}
+    else:
+        ach = nb / (avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4)}
+    roof.update({"traffic": None, "kernel": "w4a16_gemm on this rank's shard (collective excluded)",
+                 "algorithmic_per_launch": nf if prefill else nb,
+                 "peak_source": "%s (%s)" % (pk["source"], "MEASURED_PEAKS.json" if pk["source"] == "measured"
+                                             else "recipe")})
+
+    e2e = None
+    if not args.no_e2e:
+        hX = {n: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).pin_memory() for n, x in host_X.items()}
+        hY = {p.name: torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory() for _, p in plist}
+
+        def one():
+            for key, p in plist:
+                Y = layers[key].forward(hX[p.name].to(device, non_blocking=True).view(torch.bfloat16))
+                hY[p.name].copy_(Y, non_blocking=True)
+
+        one()
+        torch.cuda.synchronize()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps_e = min(args.steps, 10)
+        a0.record()
+        for _ in range(steps_e):
+            one()
+        a1.record()
+        a1.synchronize()
+        barrier()
+        e_ms, _ = aggregate(a0.elapsed_time(a1), 0.0, device)
+        e2e = {"value": round(steps_e * per_step / (e_ms * 1e-3) / (1e12 if prefill else 1e9), 2),
+               "unit": "TFLOP/s" if prefill else "GB/s",
+               "h2d_bytes_per_step": sum(x.numel() * 2 for x in hX.values()),
+               "d2h_bytes_per_step": sum(y.numel() * 2 for y in hY.values()), "steps": steps_e,
+               "what": "per rank: H2D of its activations, the sharded layer (product + collective), D2H of Y"}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s" if prefill else "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(max_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD_DESC[args.workload],
+                       "shard": "%s-split over %d ranks: %s" % (split, world, "rows of W, all-gather of Y" if split == "n"
+                                                                else "columns of W and X, all-reduce of fp32 partials, "
+                                                                     "then w4_f32_to_bf16"),
+                       "timing": "K eager steps between CUDA events on the current stream, barrier and synchronize "
+                                 "on both sides, max over ranks",
+                       "parallelism": "tp%d (%s-split)" % (world, split)},
+            "roofline": roof, "cpu_baseline": None, "e2e": e2e,
+            "gpu_launches": args.steps * len(plist) * (2 if split == "k" else 1) * world, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if pg_ok:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local_rank = dist_env()
@@ -1433,6 +1589,9 @@ def main(argv=None):
         return 0
     if args.workload in MX_WORKLOADS:
         run_mx(args, rank, world, local_rank)
+        return 0
+    if args.shard != "none":
+        run_sharded(args, rank, world, local_rank)
         return 0
     run_w4(args, rank, world, local_rank)
     return 0

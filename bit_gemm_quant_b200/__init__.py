@@ -17,6 +17,8 @@ SYM, ASYM = 0, 1
 # OR-ed into the mode of w4a16_gemm / w4a16_gemm_noalloc: the packed weight is
 # not written by the kernel right before the call on the stream (include/w4.h)
 WEIGHTS_STATIC = 0x100
+# OR-ed into the mode: Y is fp32 (the sums before their bf16 rounding)
+OUT_F32 = 0x200
 NVFP4, MXFP4 = 0, 1
 FP4_BLOCK = {NVFP4: 16, MXFP4: 32}
 MX_SCALES_ROWS, MX_SCALES_MMA = 0, 1
@@ -54,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.w4_awq_search.restype = I
         L.w4_fp4_quant.argtypes = [P, I64, I64, I, P, P, P]
         L.w4_fp4_quant.restype = I
+        L.w4_f32_to_bf16.argtypes = [P, I64, P, P]
+        L.w4_f32_to_bf16.restype = I
         L.w4_mxfp8_quant.argtypes = [P, I64, I64, P, P, I, P]
         L.w4_mxfp8_quant.restype = I
         L.w4_mx_scale_layout.argtypes = [P, I64, I64, P, P]
@@ -105,6 +109,10 @@ def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, wor
 
 def w4_fp4_quant(W, N, K, kind, codes, scales, stream) -> int:
     return lib().w4_fp4_quant(W, N, K, kind, codes, scales, stream)
+
+
+def w4_f32_to_bf16(src, n, dst, stream) -> int:
+    return lib().w4_f32_to_bf16(src, n, dst, stream)
 
 
 def w4_mxfp8_quant(X, M, K, codes, scales, scale_layout, stream) -> int:
@@ -179,17 +187,23 @@ def quant_pack(W, group: int = 128, mode: int = SYM, s=None, stream=None, out=No
 
 
 def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None, workspace=None,
-         out=None, stream=None, weights_static: bool = False):
+         out=None, stream=None, weights_static: bool = False, out_f32: bool = False):
     """Y[M,N] = X . W^T from the packed weight; X bf16 CUDA tensor [M,K].
     ``weights_static`` passes W4_WEIGHTS_STATIC: the caller declares that the
     kernel right before this call on the stream does not write the packed
     weight (weights quantized once, earlier), so the weight stream may start
-    before that kernel finishes."""
+    before that kernel finishes.  ``out_f32`` passes W4_OUT_F32: Y is fp32,
+    the sums before their bf16 rounding."""
     import torch
     M, K = X.shape
     if N is None:
         N = qweight.shape[0]
-    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if out is not None:
+        Y = out
+    else:
+        Y = torch.empty((M, N), dtype=torch.float32 if out_f32 else torch.bfloat16, device=X.device)
+    if out_f32:
+        mode |= OUT_F32
     need = w4a16_workspace_bytes(M, N, K, group)
     if need and workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=X.device)
@@ -252,6 +266,16 @@ def fp4_quant(W, kind: int = NVFP4, stream=None, out=None):
     if st != W4_OK:
         raise W4Error(st, "w4_fp4_quant")
     return codes, scales
+
+
+def f32_to_bf16(src, out=None, stream=None):
+    """bf16 (round to nearest even) copy of an fp32 CUDA tensor."""
+    import torch
+    dst = out if out is not None else torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    st = w4_f32_to_bf16(_ptr(src), src.numel(), _ptr(dst), _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_f32_to_bf16")
+    return dst
 
 
 def mx_scale_bytes(R: int, K: int) -> int:

@@ -82,6 +82,14 @@ w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *c
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+w4_status w4_f32_to_bf16(const float *src, int64_t n, void *dst, w4_stream_t stream)
+{
+    if (!src || !dst || n < 1) return W4_ERR_INVALID_ARG;
+    if (!aligned(src, 4) || !aligned(dst, 2)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e = w4::launch_f32_to_bf16(src, n, dst, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 w4_status w4_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales, int scale_layout,
                          w4_stream_t stream)
 {
@@ -145,13 +153,14 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
                      void *workspace, size_t workspace_bytes, w4_stream_t stream)
 {
     const bool weights_static = (mode & W4_WEIGHTS_STATIC) != 0;
-    mode &= ~W4_WEIGHTS_STATIC;
+    const bool y_f32 = (mode & W4_OUT_F32) != 0;
+    mode &= ~(W4_WEIGHTS_STATIC | W4_OUT_F32);
     if (!X || !qweight || !scales || !Y) return W4_ERR_INVALID_ARG;
     if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N))
         return W4_ERR_INVALID_ARG;
     if ((mode == W4_ASYM) != (qzeros != nullptr)) return W4_ERR_INVALID_ARG;
-    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(Y, 2))
+    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(Y, y_f32 ? 4 : 2))
         return W4_ERR_INVALID_ARG;
     if (qzeros && !aligned(qzeros, 4)) return W4_ERR_INVALID_ARG;
     const size_t need = w4a16_workspace_bytes(M, N, K, group);
@@ -160,10 +169,11 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
     if (!w4::gemm_shape_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
     cudaError_t e;
     if (M <= w4::kGemvMaxM)
-        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, weights_static, Y,
+        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, weights_static, y_f32, Y,
                             (cudaStream_t)stream);
     else
-        e = w4::launch_gemm_tc(X, M, N, K, qweight, scales, qzeros, group, mode, Y, workspace, (cudaStream_t)stream);
+        e = w4::launch_gemm_tc(X, M, N, K, qweight, scales, qzeros, group, mode, y_f32, Y, workspace,
+                               (cudaStream_t)stream);
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 

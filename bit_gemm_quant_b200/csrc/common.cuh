@@ -58,6 +58,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// One output element of the product: bf16 (round to nearest even) or, with
+// W4_OUT_F32, the fp32 sum itself.
+__device__ __forceinline__ void store_y(void *Y, size_t idx, float v, int y_f32)
+{
+    if (y_f32) ((float *)Y)[idx] = v;
+    else ((__nv_bfloat16 *)Y)[idx] = __float2bfloat16_rn(v);
+}
+
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -65,8 +73,8 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_fl
 cudaError_t launch_quant_pack(const void *W, int64_t N, int64_t K, int group, int mode, const float *s,
                               uint32_t *qweight, void *scales, uint32_t *qzeros, cudaStream_t stream);
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
-                        const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static, void *Y,
-                        cudaStream_t stream);
+                        const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static,
+                        bool y_f32, void *Y, cudaStream_t stream);
 // Batches up to this size run the GEMV (two MMA token groups of 8); larger ones
 // the tensor-core kernel.
 constexpr int64_t kGemvMaxM = 16;
@@ -90,6 +98,8 @@ cudaError_t set_smem_attr(Kern kern, int bytes, std::atomic<bool> (&done)[kMaxDe
 }
 cudaError_t launch_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                              cudaStream_t stream);
+// fp32 -> bf16 (round to nearest even) of n elements
+cudaError_t launch_f32_to_bf16(const float *src, int64_t n, void *dst, cudaStream_t stream);
 // MX activations, the tensor-core scale layout and the block-scaled product
 int64_t mx_padded_rows(int64_t R);
 cudaError_t launch_mxfp8_quant(const void *X, int64_t M, int64_t K, uint8_t *codes, uint8_t *scales, int layout,
@@ -102,8 +112,8 @@ size_t tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
 // byte range of the split-K tile counters inside that workspace (0 bytes if none)
 void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size_t *bytes);
 cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
-                           const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
-                           cudaStream_t stream);
+                           const void *scales, const uint32_t *qzeros, int group, int mode, bool y_f32, void *Y,
+                           void *ws, cudaStream_t stream);
 size_t awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int mode, int n_alpha);
 cudaError_t launch_awq_search(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
                               int n_alpha, double *losses, int *best, float *s_best, void *ws, cudaStream_t stream);

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, TcCfg<BN>::kMinBlocks)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_q,
                const __grid_constant__ CUtensorMap tmap_y, int y_tma, int M, int N, int K, int group_log2, int asym,
                const uint4 *__restrict__ qweight, const unsigned short *__restrict__ scales,
-               const uint32_t *__restrict__ qzeros, __nv_bfloat16 *__restrict__ Y, float *__restrict__ partial,
+               const uint32_t *__restrict__ qzeros, void *__restrict__ Y, int y_f32, float *__restrict__ partial,
                unsigned *__restrict__ counters, int splits, int kb_per_split, uint64_t wait_ns)
 {
     using C = TcCfg<BN>;
@@ -409,7 +409,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 for (int j = 0; j < CH; ++j) {
                     const int m = m0 + cbeg + c + j;
                     if (okn && m < M) {
-                        if (splits == 1) Y[(size_t)m * N + n] = __float2bfloat16_rn(acc[j]);
+                        if (splits == 1) store_y(Y, (size_t)m * N + n, acc[j], y_f32);
                         else partial[((size_t)split * M + m) * N + n] = acc[j];
                     }
                 }
@@ -446,7 +446,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                     if (okn && m < M) {
                         float sum = 0.f;
                         for (int sp = 0; sp < splits; ++sp) sum += __ldcg(partial + ((size_t)sp * M + m) * N + n);
-                        Y[(size_t)m * N + n] = __float2bfloat16_rn(sum);
+                        store_y(Y, (size_t)m * N + n, sum, y_f32);
                     }
                 }
                 if (threadIdx.x == 64) counters[blockIdx.y * gridDim.x + blockIdx.x] = 0u;
@@ -511,8 +511,8 @@ TcPlan plan_tc(int64_t M, int64_t N, int64_t K)
 template <int BN>
 cudaError_t launch_bn(const CUtensorMap &map, const CUtensorMap &qmap, const CUtensorMap &ymap, int y_tma,
                       const TcPlan &p, int M, int N, int K, int glog2, int asym,
-                      const uint32_t *qweight, const void *scales, const uint32_t *qzeros, void *Y, void *ws,
-                      cudaStream_t stream)
+                      const uint32_t *qweight, const void *scales, const uint32_t *qzeros, void *Y, int y_f32,
+                      void *ws, cudaStream_t stream)
 {
     using C = TcCfg<BN>;
     size_t smem = 1024 + C::kStages * C::kStageBytes + 256;
@@ -531,7 +531,7 @@ cudaError_t launch_bn(const CUtensorMap &map, const CUtensorMap &qmap, const CUt
     }
     dim3 grid(p.n_tiles, p.m_tiles, p.splits);
     return launch_pdl(gemm_tc_kernel<BN>, grid, dim3(kThreads), smem, stream, map, qmap, ymap, y_tma, M, N, K, glog2,
-                      asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros, (__nv_bfloat16 *)Y,
+                      asym, (const uint4 *)qweight, (const unsigned short *)scales, qzeros, Y, y_f32,
                       partial, counters, p.splits, p.kb_per_split, wait_limit_ns());
 }
 
@@ -552,8 +552,8 @@ void tc_workspace_counters(int64_t M, int64_t N, int64_t K, size_t *offset, size
 }
 
 cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
-                           const void *scales, const uint32_t *qzeros, int group, int mode, void *Y, void *ws,
-                           cudaStream_t stream)
+                           const void *scales, const uint32_t *qzeros, int group, int mode, bool y_f32, void *Y,
+                           void *ws, cudaStream_t stream)
 {
     const TcPlan p = plan_tc(M, N, K);
     EncodeTiledFn enc = encode_fn();
@@ -580,7 +580,7 @@ cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const
     // aligned; otherwise (and for split-K partials) the epilogue stores directly
     CUtensorMap ymap = map;
     int y_tma = 0;
-    if (p.splits == 1 && ((uintptr_t)Y % 16) == 0 && (N * 2) % 16 == 0) {
+    if (!y_f32 && p.splits == 1 && ((uintptr_t)Y % 16) == 0 && (N * 2) % 16 == 0) {
         const cuuint64_t ydim[2] = {(cuuint64_t)N, (cuuint64_t)M};
         const cuuint64_t ystride[1] = {(cuuint64_t)N * 2};
         const cuuint32_t ybox[2] = {128u, (cuuint32_t)p.BN};
@@ -593,11 +593,11 @@ cudaError_t launch_gemm_tc(const void *X, int64_t M, int64_t N, int64_t K, const
     const int glog2 = group == 32 ? 5 : group == 64 ? 6 : 7;
     const int asym = mode == W4_ASYM;
     switch (p.BN) {
-    case 16: return launch_bn<16>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    case 32: return launch_bn<32>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    case 64: return launch_bn<64>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    case 128: return launch_bn<128>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
-    default: return launch_bn<256>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, ws, stream);
+    case 16: return launch_bn<16>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, y_f32 ? 1 : 0, ws, stream);
+    case 32: return launch_bn<32>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, y_f32 ? 1 : 0, ws, stream);
+    case 64: return launch_bn<64>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, y_f32 ? 1 : 0, ws, stream);
+    case 128: return launch_bn<128>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, y_f32 ? 1 : 0, ws, stream);
+    default: return launch_bn<256>(map, qmap, ymap, y_tma, p, (int)M, (int)N, (int)K, glog2, asym, qweight, scales, qzeros, Y, y_f32 ? 1 : 0, ws, stream);
     }
 }
 

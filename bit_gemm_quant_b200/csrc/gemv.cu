@@ -131,7 +131,7 @@ template <int G, int MODE, int MT, int NW, int SK, int R, int MINB, bool EARLY, 
 __global__ void __launch_bounds__(NW * 32, MINB)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
-            __nv_bfloat16 *__restrict__ Y, int *err, uint64_t wait_ns)
+            void *__restrict__ Y, int y_f32, int *err, uint64_t wait_ns)
 {
     using C = GemvCfg<G, SK, NW, R, MT>;
     extern __shared__ uint8_t smem_raw[];
@@ -334,17 +334,17 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__r
                 for (int e = 0; e < 4; ++e)
                     sm[e] += ((const float(*)[4 * MT])(smem + w * R * C::kStageBytes))[lane][4 * mt + e];
             const int m0 = 8 * mt + 2 * t, m1 = m0 + 1;   // tokens of c0/c2 and c1/c3
-            if (rA < N && m0 < M) Y[(size_t)m0 * N + rA] = __float2bfloat16_rn(sm[0]);
-            if (rA < N && m1 < M) Y[(size_t)m1 * N + rA] = __float2bfloat16_rn(sm[1]);
-            if (rB < N && m0 < M) Y[(size_t)m0 * N + rB] = __float2bfloat16_rn(sm[2]);
-            if (rB < N && m1 < M) Y[(size_t)m1 * N + rB] = __float2bfloat16_rn(sm[3]);
+            if (rA < N && m0 < M) store_y(Y, (size_t)m0 * N + rA, sm[0], y_f32);
+            if (rA < N && m1 < M) store_y(Y, (size_t)m1 * N + rA, sm[1], y_f32);
+            if (rB < N && m0 < M) store_y(Y, (size_t)m0 * N + rB, sm[2], y_f32);
+            if (rB < N && m1 < M) store_y(Y, (size_t)m1 * N + rB, sm[3], y_f32);
         }
     }
 }
 
 template <int G, int MODE, int MT, int NW, int SK, int R, int MINB, bool EARLY = false, bool XPF = false>
 cudaError_t launch_cfg(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
-                       const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
+                       const uint32_t *qzeros, void *Y, int y_f32, int *err, cudaStream_t stream)
 {
     const int64_t blocks = (N + 15) / 16;             // one 16-channel tile per CTA
     constexpr int smem = GemvCfg<G, SK, NW, R, MT>::kBytes;
@@ -353,7 +353,7 @@ cudaError_t launch_cfg(const CUtensorMap &map, const void *X, int64_t M, int64_t
     const cudaError_t e = set_smem_attr(kern, smem, attr_done);
     if (e != cudaSuccess) return e;
     return launch_pdl(kern, dim3((unsigned)blocks), dim3(NW * 32), smem, stream, map, (const __nv_bfloat16 *)X,
-                      (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros, (__nv_bfloat16 *)Y, err,
+                      (int)M, (int)N, (int)K, (const unsigned short *)scales, qzeros, Y, y_f32, err,
                       wait_limit_ns());
 }
 
@@ -364,28 +364,29 @@ cudaError_t launch_cfg(const CUtensorMap &map, const void *X, int64_t M, int64_t
 // smaller ring and register budget let six CTAs share an SM.
 template <int G, int MODE, int MT, bool EARLY>
 cudaError_t launch_g(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
-                     const uint32_t *qzeros, void *Y, int *err, cudaStream_t stream)
+                     const uint32_t *qzeros, void *Y, int y_f32, int *err, cudaStream_t stream)
 {
     const int64_t tiles = (N + 15) / 16;
     if (tiles <= 2 * kNumSMs)
-        return launch_cfg<G, MODE, MT, 8, 512, 2, 2, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+        return launch_cfg<G, MODE, MT, 8, 512, 2, 2, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
     if (MT == 1 && tiles > 5 * kNumSMs && tiles <= 6 * kNumSMs)
-        return launch_cfg<G, MODE, MT, 4, 256, 2, 6, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
-    return launch_cfg<G, MODE, MT, 4, 512, 2, (MT == 1 ? 5 : 4), EARLY>(map, X, M, N, K, scales, qzeros, Y, err,
-                                                                        stream);
+        return launch_cfg<G, MODE, MT, 4, 256, 2, 6, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
+    return launch_cfg<G, MODE, MT, 4, 512, 2, (MT == 1 ? 5 : 4), EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32,
+                                                                        err, stream);
 }
 
 template <int MT, bool EARLY>
 cudaError_t launch_mt(const CUtensorMap &map, const void *X, int64_t M, int64_t N, int64_t K, const void *scales,
-                      const uint32_t *qzeros, int group, int mode, void *Y, int *err, cudaStream_t stream)
+                      const uint32_t *qzeros, int group, int mode, void *Y, int y_f32, int *err,
+                      cudaStream_t stream)
 {
     switch (group * 2 + mode) {
-    case 32 * 2 + W4_SYM: return launch_g<32, W4_SYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
-    case 32 * 2 + W4_ASYM: return launch_g<32, W4_ASYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
-    case 64 * 2 + W4_SYM: return launch_g<64, W4_SYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
-    case 64 * 2 + W4_ASYM: return launch_g<64, W4_ASYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
-    case 128 * 2 + W4_SYM: return launch_g<128, W4_SYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
-    case 128 * 2 + W4_ASYM: return launch_g<128, W4_ASYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, err, stream);
+    case 32 * 2 + W4_SYM: return launch_g<32, W4_SYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
+    case 32 * 2 + W4_ASYM: return launch_g<32, W4_ASYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
+    case 64 * 2 + W4_SYM: return launch_g<64, W4_SYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
+    case 64 * 2 + W4_ASYM: return launch_g<64, W4_ASYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
+    case 128 * 2 + W4_SYM: return launch_g<128, W4_SYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
+    case 128 * 2 + W4_ASYM: return launch_g<128, W4_ASYM, MT, EARLY>(map, X, M, N, K, scales, qzeros, Y, y_f32, err, stream);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -409,8 +410,8 @@ cudaError_t gemv_code_map(CUtensorMap *map, const uint32_t *qweight, int64_t N, 
 }
 
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
-                        const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static, void *Y,
-                        cudaStream_t stream)
+                        const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static,
+                        bool y_f32, void *Y, cudaStream_t stream)
 {
     int *err = device_error_word();
     if (!err) return cudaErrorUnknown;
@@ -418,10 +419,10 @@ cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const ui
     const cudaError_t e = gemv_code_map(&map, qweight, N, K);
     if (e != cudaSuccess) return e;
     if (M <= 8)
-        return weights_static ? launch_mt<1, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, err, stream)
-                              : launch_mt<1, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, err, stream);
-    return weights_static ? launch_mt<2, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, err, stream)
-                          : launch_mt<2, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, err, stream);
+        return weights_static ? launch_mt<1, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream)
+                              : launch_mt<1, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream);
+    return weights_static ? launch_mt<2, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream)
+                          : launch_mt<2, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream);
 }
 
 }  // namespace w4

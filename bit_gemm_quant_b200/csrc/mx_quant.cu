@@ -1,5 +1,6 @@
 // w4_mxfp8_quant: MXFP8 activations; w4_mx_scale_layout: E8M0 scales in the
-// tensor-core layout.
+// tensor-core layout; w4_f32_to_bf16: the final rounding of fp32 sums (the
+// k-split product reduces fp32 partials before it).
 //
 // Method: page 3 (blog.freezetheflame.cc quantization deep dive) section 4.3:
 // on Blackwell the FP4 weights meet activations kept at FP8, and scales are
@@ -9,7 +10,7 @@
 // e = floor(log2 amax) - 8 (8 = the exponent of E4M3's largest value 448),
 // clamped to [-127, 127]; the exact semantics are spelled out in include/w4.h.
 //
-// Both kernels are bandwidth-bound byte shuffles.  w4_mxfp8_quant gives one
+// All three kernels are bandwidth-bound elementwise passes.  w4_mxfp8_quant gives one
 // thread 8 consecutive elements (one 16-byte load, one 8-byte store); the four
 // threads of a 32-element block combine their maxima with two shuffles.  The
 // maximum is taken on the bf16 bit patterns without their sign bit (for
@@ -106,6 +107,27 @@ __global__ void __launch_bounds__(256) mx_scale_layout_kernel(const uint32_t *__
     }
 }
 
+// fp32 -> bf16, 4 elements per thread where the pointers allow it
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float *__restrict__ src, int64_t n,
+                                                          __nv_bfloat16 *__restrict__ dst, int vec)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (vec) {
+        for (int64_t i = t0; i < n / 4; i += stride) {
+            const float4 v = __ldg((const float4 *)src + i);
+            __nv_bfloat162 *d = (__nv_bfloat162 *)(dst + 4 * i);
+            d[0] = __floats2bfloat162_rn(v.x, v.y);
+            d[1] = __floats2bfloat162_rn(v.z, v.w);
+        }
+        for (int64_t i = n / 4 * 4 + t0; i < n; i += stride) dst[i] = __float2bfloat16_rn(src[i]);
+    } else {
+        for (int64_t i = t0; i < n; i += stride) dst[i] = __float2bfloat16_rn(src[i]);
+    }
+}
+
 unsigned grid_for(int64_t threads)
 {
     const int64_t want = (threads + 255) / 256;
@@ -113,6 +135,13 @@ unsigned grid_for(int64_t threads)
 }
 
 }  // namespace
+
+cudaError_t launch_f32_to_bf16(const float *src, int64_t n, void *dst, cudaStream_t stream)
+{
+    const int vec = ((uintptr_t)src % 16 == 0 && (uintptr_t)dst % 8 == 0) ? 1 : 0;
+    return launch_pdl(f32_to_bf16_kernel, dim3(grid_for(vec ? (n + 3) / 4 : n)), dim3(256), 0, stream, src, n,
+                      (__nv_bfloat16 *)dst, vec);
+}
 
 int64_t mx_padded_rows(int64_t R) { return (R + 127) / 128 * 128; }
 

@@ -58,12 +58,13 @@ bool fits(int64_t a, int64_t b) { return a > 0 && b > 0 && a <= INT64_MAX / b; }
 bool args_ok(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight, const void *scales,
              const uint32_t *qzeros, int group, int mode, const void *Y)
 {
-    mode &= ~W4_WEIGHTS_STATIC;
+    const bool f32 = (mode & W4_OUT_F32) != 0;
+    mode &= ~(W4_WEIGHTS_STATIC | W4_OUT_F32);
     if (!X || !qweight || !scales || !Y) return false;
     if (!(group == 32 || group == 64 || group == 128) || !(mode == W4_SYM || mode == W4_ASYM)) return false;
     if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N)) return false;
     if ((mode == W4_ASYM) != (qzeros != nullptr)) return false;
-    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(Y, 2)) return false;
+    if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(Y, f32 ? 4 : 2)) return false;
     if (qzeros && !aligned(qzeros, 4)) return false;
     return true;
 }

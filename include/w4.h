@@ -93,6 +93,15 @@ typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
  */
 #define W4_WEIGHTS_STATIC 0x100
 
+/*
+ * W4_OUT_F32 -- a flag OR-ed into the `mode` argument of w4a16_gemm and
+ * w4a16_gemm_noalloc: Y is fp32 [M][N] (4-byte aligned) and holds the fp32
+ * sums themselves, not their bf16 rounding.  Used by a row-parallel (k-split)
+ * product, whose partial sums are added across devices before the one bf16
+ * rounding (w4_f32_to_bf16).
+ */
+#define W4_OUT_F32 0x200
+
 /* Block-scaled FP4 kinds for w4_fp4_quant. */
 typedef enum { W4_NVFP4 = 0, W4_MXFP4 = 1 } w4_fp4_kind;
 
@@ -132,11 +141,12 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
  *   M, N, K  M >= 1, N >= 1, K % group == 0, K >= group.
  *   qweight, scales, qzeros, group, mode: as produced by w4_quant_pack
  *            (qzeros NULL in W4_SYM mode).
- *   Y        out, bf16 [M][N].
+ *   Y        out, bf16 [M][N] (fp32 [M][N], 4-byte aligned, with W4_OUT_F32).
  *   workspace, workspace_bytes: device scratch of at least
  *            w4a16_workspace_bytes(M, N, K, group) bytes (may be NULL when
  *            that is 0); 256-byte aligned.
- *   mode     W4_SYM or W4_ASYM, optionally OR-ed with W4_WEIGHTS_STATIC.
+ *   mode     W4_SYM or W4_ASYM, optionally OR-ed with W4_WEIGHTS_STATIC and
+ *            W4_OUT_F32.
  * Paths: M <= 16 runs the GEMV (codes streamed to shared memory by TMA,
  * dequantized in registers, mma.sync); larger M runs the tcgen05 kernel
  * (dequantized weights in tensor memory, activations in shared memory, fp32
@@ -237,6 +247,15 @@ w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int64_t K, con
  */
 w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                        w4_stream_t stream);
+
+/*
+ * w4_f32_to_bf16 -- dst[i] = bf16_rne(src[i]) for i < n: the one rounding of a
+ * product whose fp32 partial sums were added across devices.
+ *   src  fp32 [n], 4-byte aligned;  dst  out, bf16 [n], 2-byte aligned.
+ * Errors: W4_ERR_INVALID_ARG for NULL, misaligned or n < 1; W4_ERR_CUDA if the
+ * launch fails.  Asynchronous on `stream`.
+ */
+w4_status w4_f32_to_bf16(const float *src, int64_t n, void *dst, w4_stream_t stream);
 
 /*
  * MX scale layouts (for the E8M0 scales of w4_mxfp8_quant, w4_mx_scale_layout

@@ -183,9 +183,26 @@ def test_weights_static_flag_is_accepted_only_in_the_product_mode(w4):
     assert int(m.group(1), 16) == flag
     assert mm(w4, mode=w4.ASYM | flag) == E                  # asymmetric without qzeros: the mode was read as ASYM
     assert mm(w4, mode=w4.SYM | flag, z=FAKE) == E           # symmetric with qzeros: read as SYM
-    assert mm(w4, mode=0x200) == E                           # an unknown bit
-    assert mm(w4, mode=flag | 0x200) == E
+    assert mm(w4, mode=0x400) == E                           # an unknown bit
+    assert mm(w4, mode=flag | 0x400) == E
     assert qp(w4, mode=flag) == E                            # the quantizer has no such flag
+
+
+def test_fp32_output_flag(w4):
+    """W4_OUT_F32 is a product-mode flag like W4_WEIGHTS_STATIC; an fp32 Y must
+    be 4-byte aligned; the quantizer rejects it."""
+    E = w4.W4_ERR_INVALID_ARG
+    f32 = w4.OUT_F32
+    m = re.search(r"#define\s+W4_OUT_F32\s+(0x[0-9a-fA-F]+)", open(HEADER).read())
+    assert int(m.group(1), 16) == f32
+    assert mm(w4, mode=w4.ASYM | f32) == E                   # read as ASYM (no qzeros given)
+    assert mm(w4, mode=w4.SYM | f32 | w4.WEIGHTS_STATIC, z=FAKE) == E
+    assert mm(w4, mode=w4.SYM | f32, Y=FAKE + 2) == E        # bf16 alignment is not enough for fp32
+    assert qp(w4, mode=f32) == E
+    assert w4.w4_f32_to_bf16(None, 4, P(FAKE), None) == E
+    assert w4.w4_f32_to_bf16(P(FAKE), 0, P(FAKE), None) == E
+    assert w4.w4_f32_to_bf16(P(FAKE + 2), 4, P(FAKE), None) == E
+    assert w4.w4_f32_to_bf16(P(FAKE), 4, P(FAKE + 1), None) == E
 
 
 def test_noalloc_rejects_an_unsupported_shape_before_enqueuing_anything(w4):
