@@ -56,6 +56,10 @@ def lib() -> ctypes.CDLL:
         L.w4_awq_search.restype = I
         L.w4_fp4_quant.argtypes = [P, I64, I64, I, P, P, P]
         L.w4_fp4_quant.restype = I
+        L.w4_gptq_workspace_bytes.argtypes = [I64, I64, I]
+        L.w4_gptq_workspace_bytes.restype = SZ
+        L.w4_gptq.argtypes = [P, P, I64, I64, I64, I, I, P, P, P, P, SZ, P]
+        L.w4_gptq.restype = I
         L.w4_f32_to_bf16.argtypes = [P, I64, P, P]
         L.w4_f32_to_bf16.restype = I
         L.w4_mxfp8_quant.argtypes = [P, I64, I64, P, P, I, P]
@@ -109,6 +113,14 @@ def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, wor
 
 def w4_fp4_quant(W, N, K, kind, codes, scales, stream) -> int:
     return lib().w4_fp4_quant(W, N, K, kind, codes, scales, stream)
+
+
+def w4_gptq_workspace_bytes(N, K, group) -> int:
+    return int(lib().w4_gptq_workspace_bytes(N, K, group))
+
+
+def w4_gptq(W, X, N, K, M, group, mode, qweight, scales, qzeros, workspace, workspace_bytes, stream) -> int:
+    return lib().w4_gptq(W, X, N, K, M, group, mode, qweight, scales, qzeros, workspace, workspace_bytes, stream)
 
 
 def w4_f32_to_bf16(src, n, dst, stream) -> int:
@@ -266,6 +278,25 @@ def fp4_quant(W, kind: int = NVFP4, stream=None, out=None):
     if st != W4_OK:
         raise W4Error(st, "w4_fp4_quant")
     return codes, scales
+
+
+def gptq(W, X, group: int = 128, mode: int = SYM, stream=None):
+    """GPTQ of a bf16 CUDA tensor W[N,K] with calibration rows X[M,K] (bf16
+    CUDA); returns (qweight, scales, qzeros or None) as quant_pack does."""
+    import torch
+    N, K = W.shape
+    M = X.shape[0]
+    qs, ss, zs = packed_shapes(N, K, group)
+    qweight = torch.empty(qs, dtype=torch.int32, device=W.device)
+    scales = torch.empty(ss, dtype=torch.float16, device=W.device)
+    qzeros = torch.empty(zs, dtype=torch.int32, device=W.device) if mode == ASYM else None
+    need = w4_gptq_workspace_bytes(N, K, group)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    st = w4_gptq(_ptr(W), _ptr(X), N, K, M, group, mode, _ptr(qweight), _ptr(scales), _ptr(qzeros), _ptr(ws),
+                 ws.numel(), _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_gptq")
+    return qweight, scales, qzeros
 
 
 def f32_to_bf16(src, out=None, stream=None):

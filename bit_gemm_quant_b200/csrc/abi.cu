@@ -82,6 +82,30 @@ w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *c
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+size_t w4_gptq_workspace_bytes(int64_t N, int64_t K, int group)
+{
+    if (N < 1 || K < 32 || !group_ok(group) || K % group != 0 || K > 16384 || !fits(N, K)) return 0;
+    return w4::gptq_workspace_bytes(N, K, group);
+}
+
+w4_status w4_gptq(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
+                  uint32_t *qweight, void *scales, uint32_t *qzeros, void *workspace, size_t workspace_bytes,
+                  w4_stream_t stream)
+{
+    if (!W || !X || !qweight || !scales || !workspace) return W4_ERR_INVALID_ARG;
+    if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
+    if (N < 1 || M < 1 || K < 32 || K % group != 0 || !fits(N, K) || !fits(M, K)) return W4_ERR_INVALID_ARG;
+    if ((mode == W4_ASYM) != (qzeros != nullptr)) return W4_ERR_INVALID_ARG;
+    if (!aligned(W, 2) || !aligned(X, 2) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(workspace, 256))
+        return W4_ERR_INVALID_ARG;
+    if (qzeros && !aligned(qzeros, 4)) return W4_ERR_INVALID_ARG;
+    if (K > 16384 || N > INT32_MAX || M > INT32_MAX) return W4_ERR_UNSUPPORTED;
+    if (workspace_bytes < w4::gptq_workspace_bytes(N, K, group)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e = w4::launch_gptq(W, X, N, K, M, group, mode, qweight, scales, qzeros, workspace,
+                                          (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 w4_status w4_f32_to_bf16(const float *src, int64_t n, void *dst, w4_stream_t stream)
 {
     if (!src || !dst || n < 1) return W4_ERR_INVALID_ARG;

@@ -98,6 +98,10 @@ cudaError_t set_smem_attr(Kern kern, int bytes, std::atomic<bool> (&done)[kMaxDe
 }
 cudaError_t launch_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                              cudaStream_t stream);
+// GPTQ: workspace bytes and the whole procedure on `stream`
+size_t gptq_workspace_bytes(int64_t N, int64_t K, int group);
+cudaError_t launch_gptq(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
+                        uint32_t *qweight, void *scales, uint32_t *qzeros, void *ws, cudaStream_t stream);
 // fp32 -> bf16 (round to nearest even) of n elements
 cudaError_t launch_f32_to_bf16(const float *src, int64_t n, void *dst, cudaStream_t stream);
 // MX activations, the tensor-core scale layout and the block-scaled product

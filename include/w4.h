@@ -249,6 +249,41 @@ w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *c
                        w4_stream_t stream);
 
 /*
+ * w4_gptq_workspace_bytes -- device scratch that w4_gptq needs (0 for
+ * malformed arguments): about 16 K^2 + 8 N K bytes (the Hessian, its
+ * factor's inverse and an fp64 copy of W).
+ */
+size_t w4_gptq_workspace_bytes(int64_t N, int64_t K, int group);
+
+/*
+ * w4_gptq -- GPTQ: INT4 codes chosen column by column with Hessian-weighted
+ * error feedback, in the packed layout of w4_quant_pack (page 5 section 2.5,
+ * the column update with the upper Cholesky factor of the inverse Hessian;
+ * page 3 section 3.1, the Hessian and its damping; page 2, GPTQ section).
+ * Exact semantics (fp64 unless stated), for calibration rows X [M][K]:
+ *   H      = 2 X^T X + lambda I,  lambda = 0.01 trace(X^T X) / K
+ *   U      = upper triangular with H^-1 = U^T U  (U = I if trace(X^T X) = 0)
+ *   for j = 0 .. K-1, on every row independently:
+ *     if j % group == 0: the group's s16 and zp from fl32 of the group's
+ *        current values, by w4_quant_pack's rules (no smoothing vector)
+ *     u_j  = w4_quant_pack's code of fl32(w_j) on that grid
+ *     e    = (w_j - (u_j - zp) s16) / U[j][j];   w_k -= e U[j][k] for k > j
+ *   The result equals that definition up to the rounding order of fp64 sums
+ *   (the later columns are updated 32 columns at a time); a code can differ
+ *   only where a value lies within that rounding of a decision boundary.
+ *   W        bf16 [N][K];  X bf16 [M][K] calibration activations.
+ *   N, K, M  N >= 1, M >= 1, K >= 32, K % group == 0, K <= 16384.
+ *   group, mode, qweight, scales, qzeros: as for w4_quant_pack.
+ *   workspace, workspace_bytes: w4_gptq_workspace_bytes(N, K, group) bytes,
+ *            256-byte aligned; contents need not be initialised.
+ * About 3 K / 32 + 2 K / group kernel launches.  Errors as for w4_quant_pack;
+ * W4_ERR_UNSUPPORTED for K > 16384.  Asynchronous on `stream`.
+ */
+w4_status w4_gptq(const void *W, const void *X, int64_t N, int64_t K, int64_t M, int group, int mode,
+                  uint32_t *qweight, void *scales, uint32_t *qzeros, void *workspace, size_t workspace_bytes,
+                  w4_stream_t stream);
+
+/*
  * w4_f32_to_bf16 -- dst[i] = bf16_rne(src[i]) for i < n: the one rounding of a
  * product whose fp32 partial sums were added across devices.
  *   src  fp32 [n], 4-byte aligned;  dst  out, bf16 [n], 2-byte aligned.

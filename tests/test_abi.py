@@ -258,3 +258,23 @@ def test_mx_gemm_rejects_bad_arguments(w4):
     assert mxg(w4, Y=FAKE + 1) == E
     assert mxg(w4, flags=1) == E and mxg(w4, flags=0x300) == E   # W4_WEIGHTS_STATIC is the only flag
     assert mxg(w4, M=1 << 40, K=1 << 30) == E                 # M*K overflows int64
+
+
+def test_gptq_rejects_bad_arguments(w4):
+    E = w4.W4_ERR_INVALID_ARG
+    need = w4.w4_gptq_workspace_bytes(64, 256, 128)
+    assert need >= 16 * 256 * 256 + 8 * 64 * 256
+    assert w4.w4_gptq_workspace_bytes(64, 250, 128) == 0 and w4.w4_gptq_workspace_bytes(0, 256, 128) == 0
+    assert w4.w4_gptq_workspace_bytes(64, 32768, 128) == 0          # past the supported K
+
+    def gp(W=FAKE, X=FAKE, N=64, K=256, M=8, g=128, mode=0, q=FAKE, sc=FAKE, z=None, ws=FAKE, wsb=need):
+        return w4.w4_gptq(P(W) if W else None, P(X) if X else None, N, K, M, g, mode, P(q) if q else None,
+                          P(sc) if sc else None, P(z) if z else None, P(ws) if ws else None, wsb, None)
+    for kw in ("W", "X", "q", "sc", "ws"):
+        assert gp(**{kw: 0}) == E
+    assert gp(g=48) == E and gp(mode=2) == E
+    assert gp(N=0) == E and gp(M=0) == E and gp(K=16) == E and gp(K=320) == E
+    assert gp(mode=1) == E                        # asymmetric needs qzeros
+    assert gp(z=FAKE) == E                        # symmetric must not get qzeros
+    assert gp(ws=FAKE + 64) == E and gp(wsb=need - 1) == E
+    assert gp(W=FAKE + 1) == E and gp(q=FAKE + 2) == E
