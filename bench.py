@@ -429,6 +429,7 @@ def run_w4(args, rank, world, local_rank):
         return statistics.median(per), min(per)
 
     kt = {}
+    RP_pool = {}
     for L in launches:
         if quant_step:
             p = qp[L.label]
@@ -446,6 +447,14 @@ def run_w4(args, rank, world, local_rank):
                    for Pc in pool]
             kt[(L.name, L.label, static)] = kernel_graph_ms(fns)
         kt[(L.name, L.label)] = kt[(L.name, L.label, pp.M <= 16)]
+        if pp.M <= 16 and pp.K % 256 == 0:
+            # the same product on codes in the GEMV's box order (w4_repack, done offline)
+            if key not in RP_pool:
+                RP_pool[key] = [w4.repack(Pc[0], pp.N, pp.K) for Pc in pool]
+            fns = [(lambda Pc=Pc, Rq=Rq, pp=pp: w4.gemm(X_d[pp.name], Rq, Pc[1], Pc[2], pp.group, pp.mode, N=pp.N,
+                                                       out=Y_d[pp.name], weights_static=True, repacked=True))
+                   for Pc, Rq in zip(pool, RP_pool[key])]
+            kt[(L.name, L.label, "repacked")] = kernel_graph_ms(fns)
     torch.cuda.synchronize()
 
     step_bytes = sum(L.bytes for L in launches)
@@ -493,6 +502,12 @@ def run_w4(args, rank, world, local_rank):
             e2 = entry(L, a2, m2)
             e2["weights_static"] = False
             kernels["%s_plain[%s]" % (L.name, L.label)] = e2
+        if (L.name, L.label, "repacked") in kt:
+            a3, m3 = kt[(L.name, L.label, "repacked")]
+            e3 = entry(L, a3, m3)
+            e3["weights_static"] = True
+            e3["codes"] = "w4_repack layout (16-channel x 256-k boxes contiguous)"
+            kernels["%s_repacked[%s]" % (L.name, L.label)] = e3
         by_name.setdefault(L.name, []).append((L, [avg] * KL))
 
     dom = max(by_name, key=lambda n: sum(sum(ts) for _, ts in by_name[n]))
@@ -518,6 +533,10 @@ def run_w4(args, rank, world, local_rank):
         roof["weights_static"] = True
         plain = [kt[(L.name, L.label, False)][0] for L, _ in dom_launches]
         roof["frac_plain"] = round(per_launch / (sum(plain) / len(plain) * 1e-3) / 1e9 / pk["hbm_gbs"], 4)
+        rep = [kt.get((L.name, L.label, "repacked")) for L, _ in dom_launches]
+        if all(r is not None for r in rep):
+            roof["frac_repacked"] = round(per_launch / (sum(r[0] for r in rep) / len(rep) * 1e-3) / 1e9
+                                          / pk["hbm_gbs"], 4)
     tr = [traffic.get((dom, L.label)) for L, _ in dom_launches]
     roof["traffic"] = (sum(tr) / len(tr)) if tr and all(t is not None for t in tr) else None
     roof["kernel"] = dom

@@ -19,6 +19,8 @@ SYM, ASYM = 0, 1
 WEIGHTS_STATIC = 0x100
 # OR-ed into the mode: Y is fp32 (the sums before their bf16 rounding)
 OUT_F32 = 0x200
+# OR-ed into the mode: qweight is in the w4_repack layout (GEMV, M <= 16)
+REPACKED = 0x400
 NVFP4, MXFP4 = 0, 1
 FP4_BLOCK = {NVFP4: 16, MXFP4: 32}
 MX_SCALES_ROWS, MX_SCALES_MMA = 0, 1
@@ -56,6 +58,10 @@ def lib() -> ctypes.CDLL:
         L.w4_awq_search.restype = I
         L.w4_fp4_quant.argtypes = [P, I64, I64, I, P, P, P]
         L.w4_fp4_quant.restype = I
+        L.w4_repacked_words.argtypes = [I64, I64]
+        L.w4_repacked_words.restype = SZ
+        L.w4_repack.argtypes = [P, I64, I64, P, P]
+        L.w4_repack.restype = I
         L.w4_gptq_workspace_bytes.argtypes = [I64, I64, I]
         L.w4_gptq_workspace_bytes.restype = SZ
         L.w4_gptq.argtypes = [P, P, I64, I64, I64, I, I, P, P, P, P, SZ, P]
@@ -113,6 +119,14 @@ def w4_awq_search(W, X, N, K, M, group, mode, n_alpha, losses, best, s_best, wor
 
 def w4_fp4_quant(W, N, K, kind, codes, scales, stream) -> int:
     return lib().w4_fp4_quant(W, N, K, kind, codes, scales, stream)
+
+
+def w4_repacked_words(N, K) -> int:
+    return int(lib().w4_repacked_words(N, K))
+
+
+def w4_repack(qweight, N, K, out, stream) -> int:
+    return lib().w4_repack(qweight, N, K, out, stream)
 
 
 def w4_gptq_workspace_bytes(N, K, group) -> int:
@@ -199,16 +213,20 @@ def quant_pack(W, group: int = 128, mode: int = SYM, s=None, stream=None, out=No
 
 
 def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None, workspace=None,
-         out=None, stream=None, weights_static: bool = False, out_f32: bool = False):
+         out=None, stream=None, weights_static: bool = False, out_f32: bool = False, repacked: bool = False):
     """Y[M,N] = X . W^T from the packed weight; X bf16 CUDA tensor [M,K].
     ``weights_static`` passes W4_WEIGHTS_STATIC: the caller declares that the
     kernel right before this call on the stream does not write the packed
     weight (weights quantized once, earlier), so the weight stream may start
     before that kernel finishes.  ``out_f32`` passes W4_OUT_F32: Y is fp32,
-    the sums before their bf16 rounding."""
+    the sums before their bf16 rounding.  ``repacked`` passes W4_REPACKED:
+    qweight comes from ``repack`` (give N then, the padded array has more
+    rows)."""
     import torch
     M, K = X.shape
     if N is None:
+        if repacked:
+            raise ValueError("gemm(repacked=True) needs N: the repacked array's shape does not give it")
         N = qweight.shape[0]
     if out is not None:
         Y = out
@@ -216,6 +234,8 @@ def gemm(X, qweight, scales, qzeros, group: int, mode: int, N: int | None = None
         Y = torch.empty((M, N), dtype=torch.float32 if out_f32 else torch.bfloat16, device=X.device)
     if out_f32:
         mode |= OUT_F32
+    if repacked:
+        mode |= REPACKED
     need = w4a16_workspace_bytes(M, N, K, group)
     if need and workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=X.device)
@@ -278,6 +298,18 @@ def fp4_quant(W, kind: int = NVFP4, stream=None, out=None):
     if st != W4_OK:
         raise W4Error(st, "w4_fp4_quant")
     return codes, scales
+
+
+def repack(qweight, N: int, K: int, stream=None, out=None):
+    """The GEMV's box order of a packed weight (int32 [N, K/8] CUDA tensor):
+    a flat int32 tensor of w4_repacked_words(N, K) words."""
+    import torch
+    n = w4_repacked_words(N, K)
+    dst = out if out is not None else torch.empty(max(n, 4), dtype=torch.int32, device=qweight.device)
+    st = w4_repack(_ptr(qweight), N, K, _ptr(dst), _stream_handle(stream))
+    if st != W4_OK:
+        raise W4Error(st, "w4_repack")
+    return dst
 
 
 def gptq(W, X, group: int = 128, mode: int = SYM, stream=None):

@@ -82,6 +82,22 @@ w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *c
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+size_t w4_repacked_words(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 256 || K % 256 != 0 || !fits(N + 15, K)) return 0;
+    return (size_t)((N + 15) / 16 * 16) * (size_t)(K / 8);
+}
+
+w4_status w4_repack(const uint32_t *qweight, int64_t N, int64_t K, uint32_t *out, w4_stream_t stream)
+{
+    if (!qweight || !out) return W4_ERR_INVALID_ARG;
+    if (N < 1 || K < 256 || !fits(N + 15, K)) return W4_ERR_INVALID_ARG;
+    if (K % 256 != 0) return W4_ERR_UNSUPPORTED;
+    if (!aligned(qweight, 16) || !aligned(out, 16)) return W4_ERR_INVALID_ARG;
+    const cudaError_t e = w4::launch_repack(qweight, N, K, out, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 size_t w4_gptq_workspace_bytes(int64_t N, int64_t K, int group)
 {
     if (N < 1 || K < 32 || !group_ok(group) || K % group != 0 || K > 16384 || !fits(N, K)) return 0;
@@ -178,7 +194,8 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
 {
     const bool weights_static = (mode & W4_WEIGHTS_STATIC) != 0;
     const bool y_f32 = (mode & W4_OUT_F32) != 0;
-    mode &= ~(W4_WEIGHTS_STATIC | W4_OUT_F32);
+    const bool repacked = (mode & W4_REPACKED) != 0;
+    mode &= ~(W4_WEIGHTS_STATIC | W4_OUT_F32 | W4_REPACKED);
     if (!X || !qweight || !scales || !Y) return W4_ERR_INVALID_ARG;
     if (!group_ok(group) || !mode_ok(mode)) return W4_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N))
@@ -191,9 +208,10 @@ w4_status w4a16_gemm(const void *X, int64_t M, int64_t N, int64_t K, const uint3
     if (need > workspace_bytes || (need > 0 && (!workspace || !aligned(workspace, 256))))
         return W4_ERR_INVALID_ARG;
     if (!w4::gemm_shape_supported(M, N, K)) return W4_ERR_UNSUPPORTED;
+    if (repacked && (M > w4::kGemvMaxM || K % 256 != 0)) return W4_ERR_UNSUPPORTED;
     cudaError_t e;
     if (M <= w4::kGemvMaxM)
-        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, weights_static, y_f32, Y,
+        e = w4::launch_gemv(X, M, N, K, qweight, scales, qzeros, group, mode, weights_static, y_f32, repacked, Y,
                             (cudaStream_t)stream);
     else
         e = w4::launch_gemm_tc(X, M, N, K, qweight, scales, qzeros, group, mode, y_f32, Y, workspace,

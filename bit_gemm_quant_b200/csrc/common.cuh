@@ -74,7 +74,9 @@ cudaError_t launch_quant_pack(const void *W, int64_t N, int64_t K, int group, in
                               uint32_t *qweight, void *scales, uint32_t *qzeros, cudaStream_t stream);
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                         const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static,
-                        bool y_f32, void *Y, cudaStream_t stream);
+                        bool y_f32, bool repacked, void *Y, cudaStream_t stream);
+// the GEMV's code layout: w4_repack (16-row x 256-k boxes stored contiguously)
+cudaError_t launch_repack(const uint32_t *qweight, int64_t N, int64_t K, uint32_t *out, cudaStream_t stream);
 // Batches up to this size run the GEMV (two MMA token groups of 8); larger ones
 // the tensor-core kernel.
 constexpr int64_t kGemvMaxM = 16;

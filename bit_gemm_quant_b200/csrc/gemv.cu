@@ -131,8 +131,12 @@ template <int G, int MODE, int MT, int NW, int SK, int R, int MINB, bool EARLY, 
 __global__ void __launch_bounds__(NW * 32, MINB)
 gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__restrict__ X, int M, int N, int K,
             const unsigned short *__restrict__ scales, const uint32_t *__restrict__ qzeros,
-            void *__restrict__ Y, int y_f32, int *err, uint64_t wait_ns)
+            void *__restrict__ Y, int yflags, int *err, uint64_t wait_ns)
 {
+    // bit 0: fp32 Y (W4_OUT_F32); bit 1: codes in the repacked layout
+    // (w4_repack: 2 KB boxes stored contiguously, the tensor map is 4-D)
+    const int y_f32 = yflags & 1;
+    const bool repacked = (yflags & 2) != 0;
     using C = GemvCfg<G, SK, NW, R, MT>;
     extern __shared__ uint8_t smem_raw[];
     // (an offset from the shared array, not an integer cast, so that the
@@ -176,12 +180,20 @@ gemv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __nv_bfloat16 *__r
                      "r"(C::kStageBytes)
                      : "memory");
 #pragma unroll
-        for (int bb = 0; bb < C::kBoxes; ++bb)        // a box past the end of K is zero-filled
-            asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-                "[%2];" ::"r"(ring_s + s * C::kStageBytes + bb * C::kBoxBytes),
-                "l"(&tmap_q), "r"(bar0 + 8 * s), "r"((sb * C::kBoxes + bb) * 32), "r"(r0)
-                : "memory");
+        for (int bb = 0; bb < C::kBoxes; ++bb) {      // a box past the end of K is zero-filled
+            if (repacked)
+                asm volatile(
+                    "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %3, "
+                    "%4, %5}], [%2];" ::"r"(ring_s + s * C::kStageBytes + bb * C::kBoxBytes),
+                    "l"(&tmap_q), "r"(bar0 + 8 * s), "r"(0), "r"(sb * C::kBoxes + bb), "r"(r0 >> 4)
+                    : "memory");
+            else
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+                    "%4}], [%2];" ::"r"(ring_s + s * C::kStageBytes + bb * C::kBoxBytes),
+                    "l"(&tmap_q), "r"(bar0 + 8 * s), "r"((sb * C::kBoxes + bb) * 32), "r"(r0)
+                    : "memory");
+        }
     };
     if (lane == 0)
         for (int i = 0; i < R && i < nsw; ++i) issue(i);
@@ -394,35 +406,77 @@ cudaError_t launch_mt(const CUtensorMap &map, const void *X, int64_t M, int64_t 
 }  // namespace
 
 // The codes as a 2-D array of 32-bit words [N][K/8]; one box = 16 channels x
-// 32 words (256 k) with the 128-byte swizzle.
-cudaError_t gemv_code_map(CUtensorMap *map, const uint32_t *qweight, int64_t N, int64_t K)
+// 32 words (256 k) with the 128-byte swizzle.  Repacked codes (w4_repack) are
+// the same boxes stored one after another: a 4-D array [ceil(N/16)][K/256][16]
+// [32 words] whose box {32, 16, 1, 1} lands in shared memory exactly as the
+// 2-D box does; a box at k-chunk K/256 or past it is out of range and
+// zero-filled, as in the 2-D map.
+cudaError_t gemv_code_map(CUtensorMap *map, const uint32_t *qweight, int64_t N, int64_t K, bool repacked)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t gdim[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
-    const cuuint64_t gstride[1] = {(cuuint64_t)K / 2};
-    const cuuint32_t box[2] = {32u, 16u};
-    const cuuint32_t estride[2] = {1u, 1u};
-    const CUresult cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(qweight), gdim, gstride,
-                            box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult cr;
+    if (repacked) {
+        const cuuint64_t gdim[4] = {32u, 16u, (cuuint64_t)(K / 256), (cuuint64_t)((N + 15) / 16)};
+        const cuuint64_t gstride[3] = {128u, 2048u, (cuuint64_t)(K / 256) * 2048u};
+        const cuuint32_t box[4] = {32u, 16u, 1u, 1u};
+        const cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+        cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint32_t *>(qweight), gdim, gstride, box, estride,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        const cuuint64_t gdim[2] = {(cuuint64_t)(K / 8), (cuuint64_t)N};
+        const cuuint64_t gstride[1] = {(cuuint64_t)K / 2};
+        const cuuint32_t box[2] = {32u, 16u};
+        const cuuint32_t estride[2] = {1u, 1u};
+        cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(qweight), gdim, gstride, box, estride,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     return cr == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// w4_repack: dst word (((n/16) * (K/256) + kw/32) * 16 + n%16) * 32 + kw%32 =
+// qweight[n][kw] (0 for the rows that pad N to a multiple of 16); one thread
+// per 4 words.
+__global__ void __launch_bounds__(256) repack_kernel(const uint4 *__restrict__ q, int64_t N, int64_t K,
+                                                     uint4 *__restrict__ out)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t KW = K / 8, KC = K / 256;
+    const int64_t total = (N + 15) / 16 * 16 * KW / 4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t w = i * 4;                           // first destination word
+        const int64_t box = w / 512, in = w % 512;         // 16 rows x 32 words per box
+        const int64_t t = box / KC, c = box % KC;
+        const int64_t n = t * 16 + in / 32, kw = c * 32 + in % 32;
+        out[i] = n < N ? __ldg(q + (n * KW + kw) / 4) : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+cudaError_t launch_repack(const uint32_t *qweight, int64_t N, int64_t K, uint32_t *out, cudaStream_t stream)
+{
+    const int64_t threads = (N + 15) / 16 * 16 * (K / 8) / 4;
+    const int64_t want = (threads + 255) / 256;
+    const unsigned grid = (unsigned)(want < (int64_t)kNumSMs * 16 ? (want > 0 ? want : 1) : (int64_t)kNumSMs * 16);
+    return launch_pdl(repack_kernel, dim3(grid), dim3(256), 0, stream, (const uint4 *)qweight, N, K, (uint4 *)out);
 }
 
 cudaError_t launch_gemv(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qweight,
                         const void *scales, const uint32_t *qzeros, int group, int mode, bool weights_static,
-                        bool y_f32, void *Y, cudaStream_t stream)
+                        bool y_f32, bool repacked, void *Y, cudaStream_t stream)
 {
     int *err = device_error_word();
     if (!err) return cudaErrorUnknown;
     CUtensorMap map;
-    const cudaError_t e = gemv_code_map(&map, qweight, N, K);
+    const cudaError_t e = gemv_code_map(&map, qweight, N, K, repacked);
     if (e != cudaSuccess) return e;
     if (M <= 8)
-        return weights_static ? launch_mt<1, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream)
-                              : launch_mt<1, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream);
-    return weights_static ? launch_mt<2, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream)
-                          : launch_mt<2, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, y_f32 ? 1 : 0, err, stream);
+        return weights_static ? launch_mt<1, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, (y_f32 ? 1 : 0) | (repacked ? 2 : 0), err, stream)
+                              : launch_mt<1, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, (y_f32 ? 1 : 0) | (repacked ? 2 : 0), err, stream);
+    return weights_static ? launch_mt<2, true>(map, X, M, N, K, scales, qzeros, group, mode, Y, (y_f32 ? 1 : 0) | (repacked ? 2 : 0), err, stream)
+                          : launch_mt<2, false>(map, X, M, N, K, scales, qzeros, group, mode, Y, (y_f32 ? 1 : 0) | (repacked ? 2 : 0), err, stream);
 }
 
 }  // namespace w4

@@ -59,7 +59,7 @@ bool args_ok(const void *X, int64_t M, int64_t N, int64_t K, const uint32_t *qwe
              const uint32_t *qzeros, int group, int mode, const void *Y)
 {
     const bool f32 = (mode & W4_OUT_F32) != 0;
-    mode &= ~(W4_WEIGHTS_STATIC | W4_OUT_F32);
+    mode &= ~(W4_WEIGHTS_STATIC | W4_OUT_F32 | W4_REPACKED);
     if (!X || !qweight || !scales || !Y) return false;
     if (!(group == 32 || group == 64 || group == 128) || !(mode == W4_SYM || mode == W4_ASYM)) return false;
     if (M < 1 || N < 1 || K < group || K % group != 0 || !fits(M, K) || !fits(N, K) || !fits(M, N)) return false;

@@ -102,6 +102,15 @@ typedef enum { W4_SYM = 0, W4_ASYM = 1 } w4_mode;
  */
 #define W4_OUT_F32 0x200
 
+/*
+ * W4_REPACKED -- a flag OR-ed into the `mode` argument of w4a16_gemm and
+ * w4a16_gemm_noalloc: `qweight` is in the layout that w4_repack writes (the
+ * GEMV's 16-channel x 256-k boxes stored one after another), not the canonical
+ * [N][K/8].  The codes are the same, and so is every bit of Y.  Served by the
+ * GEMV only: M <= 16 and K % 256 == 0, else W4_ERR_UNSUPPORTED.
+ */
+#define W4_REPACKED 0x400
+
 /* Block-scaled FP4 kinds for w4_fp4_quant. */
 typedef enum { W4_NVFP4 = 0, W4_MXFP4 = 1 } w4_fp4_kind;
 
@@ -145,8 +154,8 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K, int group);
  *   workspace, workspace_bytes: device scratch of at least
  *            w4a16_workspace_bytes(M, N, K, group) bytes (may be NULL when
  *            that is 0); 256-byte aligned.
- *   mode     W4_SYM or W4_ASYM, optionally OR-ed with W4_WEIGHTS_STATIC and
- *            W4_OUT_F32.
+ *   mode     W4_SYM or W4_ASYM, optionally OR-ed with W4_WEIGHTS_STATIC,
+ *            W4_OUT_F32 and W4_REPACKED.
  * Paths: M <= 16 runs the GEMV (codes streamed to shared memory by TMA,
  * dequantized in registers, mma.sync); larger M runs the tcgen05 kernel
  * (dequantized weights in tensor memory, activations in shared memory, fp32
@@ -247,6 +256,28 @@ w4_status w4a16_gemm_noalloc(const void *X, int64_t M, int64_t N, int64_t K, con
  */
 w4_status w4_fp4_quant(const void *W, int64_t N, int64_t K, int kind, uint8_t *codes, uint8_t *scales,
                        w4_stream_t stream);
+
+/*
+ * w4_repacked_words -- 32-bit words of the repacked layout of an [N][K/8]
+ * packed weight: ceil(N/16) * 16 * K/8 (0 unless K % 256 == 0).
+ */
+size_t w4_repacked_words(int64_t N, int64_t K);
+
+/*
+ * w4_repack -- the offline repack of a packed weight into the GEMV's box
+ * order (a layout-specialised copy in the spirit of page 3 section 3.1's
+ * Marlin, which reorders INT4 weights offline into the tiles its kernel
+ * reads; the codes themselves are unchanged).  Word kw of channel n goes to
+ *   (((n/16) * (K/256) + kw/32) * 16 + n % 16) * 32 + kw % 32,
+ * so that each 16-channel x 256-k box the GEMV loads is 2 KB of contiguous
+ * memory; the channels that pad N to a multiple of 16 are written as 0.
+ *   qweight  uint32 [N][K/8] (w4_quant_pack layout), 16-byte aligned.
+ *   N, K     N >= 1, K >= 256; K % 256 != 0 gives W4_ERR_UNSUPPORTED.
+ *   out      out, w4_repacked_words(N, K) words, 16-byte aligned; scales and
+ *            zero-points keep their layout.
+ * Errors as for w4_quant_pack.  Asynchronous on `stream`.
+ */
+w4_status w4_repack(const uint32_t *qweight, int64_t N, int64_t K, uint32_t *out, w4_stream_t stream);
 
 /*
  * w4_gptq_workspace_bytes -- device scratch that w4_gptq needs (0 for

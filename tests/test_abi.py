@@ -183,8 +183,8 @@ def test_weights_static_flag_is_accepted_only_in_the_product_mode(w4):
     assert int(m.group(1), 16) == flag
     assert mm(w4, mode=w4.ASYM | flag) == E                  # asymmetric without qzeros: the mode was read as ASYM
     assert mm(w4, mode=w4.SYM | flag, z=FAKE) == E           # symmetric with qzeros: read as SYM
-    assert mm(w4, mode=0x400) == E                           # an unknown bit
-    assert mm(w4, mode=flag | 0x400) == E
+    assert mm(w4, mode=0x800) == E                           # an unknown bit
+    assert mm(w4, mode=flag | 0x800) == E
     assert qp(w4, mode=flag) == E                            # the quantizer has no such flag
 
 
@@ -278,3 +278,17 @@ def test_gptq_rejects_bad_arguments(w4):
     assert gp(z=FAKE) == E                        # symmetric must not get qzeros
     assert gp(ws=FAKE + 64) == E and gp(wsb=need - 1) == E
     assert gp(W=FAKE + 1) == E and gp(q=FAKE + 2) == E
+
+
+def test_repack_arguments(w4):
+    assert w4.w4_repacked_words(4096, 4096) == 4096 * 512
+    assert w4.w4_repacked_words(1000, 4096) == 1008 * 512        # N padded to whole 16-channel boxes
+    assert w4.w4_repacked_words(16, 384) == 0                    # K not a multiple of 256
+    E, U = w4.W4_ERR_INVALID_ARG, w4.W4_ERR_UNSUPPORTED
+    rp = lambda q=FAKE, N=16, K=512, out=FAKE: w4.w4_repack(P(q) if q else None, N, K, P(out) if out else None, None)
+    assert rp(q=0) == E and rp(out=0) == E and rp(N=0) == E and rp(K=128) == E
+    assert rp(K=384) == U
+    assert rp(q=FAKE + 4) == E and rp(out=FAKE + 8) == E
+    # the repacked layout is served by the GEMV only, with whole 256-k boxes
+    assert mm(w4, K=384, g=128, mode=w4.REPACKED) == U
+    assert mm(w4, mode=w4.REPACKED | 0x800) == E
