@@ -153,7 +153,9 @@ def check_product(w4, X_bits, W_bits, what):
 # activation tile width (16, 32, 64, 128, 256 tokens); two 256-token tiles
 # whose second reaches into a partial 128-row scale band; split k
 SHAPES = [(3, 128, 128), (4, 256, 512), (1, 300, 384), (20, 700, 1024), (64, 256, 2048), (100, 384, 512),
-          (200, 256, 1024), (300, 130, 640), (1, 4096, 4096), (16, 1000, 2048)]
+          (200, 256, 1024), (300, 130, 640), (1, 4096, 4096), (16, 1000, 2048),
+          # single tiles and few k-stages, many tiles with long k, the decode widths
+          (1, 128, 256), (2, 1024, 1024), (9, 8192, 512), (16, 11008, 4096)]
 
 
 @pytest.mark.gpu
