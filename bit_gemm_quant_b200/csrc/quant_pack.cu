@@ -23,28 +23,28 @@
 //     next as soon as its lanes have read an item; other rows are read with
 //     four 32-byte loads per lane, the item two steps ahead asked into L2
 //     (cp.async.bulk.prefetch);
-//   * group amax / min / max: packed bf16x2 min and max over the lane's raw
-//     words (fp32 comparisons after the fold) and at most one
-//     __shfl_xor_sync; the per-group IEEE divisions (scale and zero point)
-//     and the reciprocal are amortized over 64 weights per lane;
+//   * group amax / min / max: one packed bf16x2 max-of-magnitudes (symmetric)
+//     or a min and a max (asymmetric) per raw word (fp32 comparisons after
+//     the fold) and at most one __shfl_xor_sync; the per-group IEEE
+//     division of the scale and the reciprocal are amortized over 64
+//     weights per lane;
 //   * with a fold, the 64 weights are folded once per item (w' = fl32(w * s))
 //     and kept as fp32 pairs; the smoothing vector is staged once per CTA in
 //     shared memory, each 64-factor slice rotated by (slice % 8) float4 so
 //     that the lanes' reads of their slices (256 bytes apart) do not collide
 //     on banks, and the weights are read past L1 so that it keeps s;
-//   * per weight the code is rint(w'/s16) with IEEE semantics.  The fast path
-//     adds the magic constant 1.5*2^23 + zp to w' * rcp(s16), which leaves
-//     0x4B400000 + u in the float's bits, and computes the exact residual
-//     rho = w' - r * s16 (Sterbenz: r * s16 has <= 16 significant bits), two
-//     weights per fma/add instruction.  A packed word (8 weights) whose
-//     largest |rho| reaches s16/2 -- an exact tie of the quotient (common
-//     with bf16 weights) or a rounding the approximation got wrong -- is
-//     flagged and recomputed exactly from its raw weights, read again from
-//     cache (ties to even); groups whose fp16 scale saturated or is subnormal
-//     take an IEEE-division path;
-//   * y is monotonic in w', so the asymmetric clamp to [0, 15] (needed before
-//     packing: a code of -1 or 16 would borrow from or carry into the next
-//     nibble) runs only in warps where some group's extremes map outside;
+//   * per weight the code is rint(w'/s16) with IEEE semantics (ties to
+//     even): t1 = t0 + (w' - t0 * s16) * rcp(s16), t0 = w' * rcp(s16) -- one
+//     correction step, the residual exact -- rounds exactly like w'/s16,
+//     ties included, for bf16 and folded fp32 weights alike (see quot2), and
+//     adding the magic constant 1.5*2^23 leaves 0x4B400000 + rint(t1) in the
+//     float's bits (then + zp), two weights per fma/mul/add instruction and
+//     no check or fix-up pass.  Groups whose fp16 scale saturated or is
+//     subnormal (codes that need clamping) take an IEEE-division path;
+//   * the code is monotonic in w', so the asymmetric clamp to [0, 15]
+//     (needed before packing: a code of -1 or 16 would borrow from or carry
+//     into the next nibble) runs only in warps where some group's extremes
+//     map outside;
 //   * packing: with bits(y) = C + u (C's low byte 0), one IMAD y_b*16 + y_a
 //     puts the byte u_a | u_b << 4 in the low byte; three PRMTs assemble the
 //     word (even elements in the low half-word), and each lane stores its 8
@@ -62,9 +62,7 @@ namespace {
 // 1.5 * 2^23: for |t| < 2^22, fl32(t + kMagic) has rint(t) in its low mantissa
 // bits, because the spacing of floats in [2^23, 2^24) is 1.
 constexpr float kMagic = 12582912.0f;
-// rcp.approx is within 2 ulp of 1/s16, so w' * rcp(s16) is within
-// |w'/s16| * 2^-22 <= 2^-18 of the exact quotient: a rounding it gets wrong
-// leaves a residual of at least half a step, which the exact check catches.
+// rcp.approx is within 2 ulp of 1/s16 (quot2 corrects the quotient it gives).
 __device__ __forceinline__ float rcp_approx(float d)
 {
     float r;
@@ -121,6 +119,40 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b)
     return d;
 }
 
+// Per half: the larger of |a| and |b| in magnitude (its sign bit is not used).
+__device__ __forceinline__ uint32_t bmaxabs2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// The quotient x / d (d > 0 an fp16 value, or d = 0 with inv = 0) for rint:
+// t0 = fl(x * inv) with inv = rcp.approx(d) (within 2 ulp of 1/d) is within
+// |x/d| * 2^-21 of q = x/d; the residual x - t0 * d is a multiple of
+// ulp(t0) * ulp(d) below 2^15 of them, so the fma gives it exactly; and
+// t1 = fl(t0 + e * inv) is q + (q - t0) * (d * inv - 1) rounded once, i.e.
+// within |q| * 2^-42 + half an ulp of q.  For x an fp32 value (a bf16 weight
+// or a folded one) and q < 2^11, a half-integer h other than q is farther
+// from q than half an ulp of q by at least |q| * 2^-36: x - h * d is a
+// nonzero multiple of ulp(x), and ulp(x) / d exceeds half an ulp of q by
+// that much because d < 2^(e+1) - ulp(d) for d in [2^e, 2^(e+1)).  So t1 lies
+// on q's side of every half-integer, and t1 = h exactly when q = h: rint(t1)
+// = rint(q), ties included.
+__device__ __forceinline__ float2 quot2(float2 x, float2 inv2, float2 nd2)
+{
+    const float2 t0 = __fmul2_rn(x, inv2);
+    const float2 e = __ffma2_rn(t0, nd2, x);
+    return __ffma2_rn(e, inv2, t0);
+}
+
+__device__ __forceinline__ float quot(float x, float inv, float d)
+{
+    const float t0 = __fmul_rn(x, inv);
+    const float e = __fmaf_rn(-t0, d, x);
+    return __fmaf_rn(e, inv, t0);
+}
+
 // The two weights of raw word v (elements 2p and 2p+1 of the lane), folded.
 template <bool FOLD>
 __device__ __forceinline__ float2 weight_pair(uint32_t v, float2 sp)
@@ -131,43 +163,35 @@ __device__ __forceinline__ float2 weight_pair(uint32_t v, float2 sp)
 
 // Per-group parameters of the fast path.
 struct QParams {
-    float inv, magic, d, hd, ymax;
+    float inv, magic, d, ymax;
     int zp;
 };
 
-// Fast-path codes of one 32-weight chunk (16 raw words): y = fl(w' * rcp(s16)
-// + magic) holds r + zp (or r + 8) in its low bits, r = rint of the
-// approximate quotient; rho = w' - r * s16 is exact.  Bit w of the returned
-// flags marks packed word w (8 weights) if any of its residuals reaches half a
-// step (|rho| >= s16 / 2): exact ties of the quotient and roundings the
-// approximation got wrong.  With CLAMP the asymmetric codes are clamped to
-// [0, 15] after the residual is taken and before packing (a code of -1 or 16
-// would borrow from or carry into the neighbouring nibble); without it the
-// caller has shown that every y lies in range.  The arithmetic runs on pairs (fma / add of two fp32 lanes per
-// instruction, each correctly rounded).  With FOLD, xf holds the chunk's 16
-// folded weight pairs (w * s in fp32) and cur is not read.
+// Codes of one 32-weight chunk (16 raw words, or with FOLD the chunk's 16
+// folded weight pairs xf, w * s in fp32, and cur is not read): y = fl(t1 +
+// magic) holds rint(t1) + zp (or + 8) in its low bits, t1 the corrected
+// quotient of quot2, which rounds exactly like w'/s16; for asymmetric groups
+// zp is added after the rounding (a tie rounds to even before the shift, as
+// rint(w'/s16) + zp asks).  With CLAMP the asymmetric codes are clamped to
+// [0, 15] before packing (a code of -1 or 16 would borrow from or carry into
+// the neighbouring nibble); without it the caller has shown that every y
+// lies in range.  The arithmetic runs on pairs (fma / mul / add of two fp32
+// lanes per instruction, each correctly rounded).
 template <int MODE, bool FOLD, bool CLAMP>
-__device__ __forceinline__ uint32_t encode(const uint32_t *cur, const float2 *xf, const QParams &q,
-                                           uint32_t (&wd)[4])
+__device__ __forceinline__ void encode(const uint32_t *cur, const float2 *xf, const QParams &q, uint32_t (&wd)[4])
 {
-    const float2 inv2 = make_float2(q.inv, q.inv), mg2 = make_float2(q.magic, q.magic);
-    const float2 nmg2 = make_float2(-q.magic, -q.magic), nd2 = make_float2(-q.d, -q.d);
-    uint32_t flags = 0u;
+    const float2 inv2 = make_float2(q.inv, q.inv), nd2 = make_float2(-q.d, -q.d);
+    const float k = (MODE == W4_SYM) ? q.magic : kMagic;   // + 8 is even: a tie rounds the same way
+    const float2 k2 = make_float2(k, k), z2 = make_float2((float)q.zp, (float)q.zp);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
         uint32_t yb[8];
-        float m = 0.f;                           // largest |rho| of the word
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int p = 4 * w + j;
             const float2 x = FOLD ? xf[p] : weight_pair<false>(cur[p], make_float2(1.f, 1.f));
-            float2 y = __ffma2_rn(x, inv2, mg2);
-            // the residual of the unclamped rounding: clip(rint(w'/s16) + zp)
-            // only needs rint itself to be exact, so a weight that the clamp
-            // moves (the group maximum may round to 16) is not flagged
-            const float2 r = __fadd2_rn(y, nmg2);
-            const float2 rho = __ffma2_rn(r, nd2, x);
-            m = fmaxf(m, fmaxf(fabsf(rho.x), fabsf(rho.y)));
+            float2 y = __fadd2_rn(quot2(x, inv2, nd2), k2);
+            if (MODE == W4_ASYM) y = __fadd2_rn(y, z2);
             if (MODE == W4_ASYM && CLAMP) {
                 y.x = fmaxf(fminf(y.x, q.ymax), kMagic);
                 y.y = fmaxf(fminf(y.y, q.ymax), kMagic);
@@ -175,27 +199,8 @@ __device__ __forceinline__ uint32_t encode(const uint32_t *cur, const float2 *xf
             yb[2 * j] = __float_as_uint(y.x);
             yb[2 * j + 1] = __float_as_uint(y.y);
         }
-        if (m >= q.hd) flags |= 1u << w;
         wd[w] = pack_word(yb);
     }
-    return flags;
-}
-
-// The exact code of one weight (its fast-path y recomputed, then the tie or
-// the wrong rounding resolved from the exact residual).
-template <int MODE>
-__device__ __forceinline__ uint32_t exact_code(float x, const QParams &q)
-{
-    float y = __fmaf_rn(x, q.inv, q.magic);
-    if (MODE == W4_ASYM) y = fmaxf(fminf(y, q.ymax), kMagic);
-    const float r = __fsub_rn(y, q.magic);
-    const float rho = __fmaf_rn(-r, q.d, x);
-    const float ar = fabsf(rho);
-    // beyond half a step, or an exact tie with r odd: one step toward rho
-    const int odd = (int)(__float_as_uint(y) ^ (uint32_t)q.zp) & 1;
-    int c = (int)r;
-    if (ar > q.hd || (ar == q.hd && odd)) c += (rho > 0.f) ? 1 : -1;
-    return (MODE == W4_SYM) ? (uint32_t)(min(max(c, -8), 7) + 8) : (uint32_t)min(max(c + q.zp, 0), 15);
 }
 
 // The code of one weight by IEEE division (groups whose fp16 scale saturated
@@ -208,30 +213,52 @@ __device__ __forceinline__ uint32_t division_code(float x, const QParams &q)
                             : (uint32_t)(int)fminf(fmaxf(c + (float)q.zp, 0.f), 15.f);
 }
 
+// fl32(v / c) for c = 7 or 15 without a division: q0 = v * rc (rc = fl32(1/c)),
+// the residual v - q0 * c exactly by an fma, and one correction step.  For
+// these two divisors the result is correctly rounded for every one of the 2^23
+// significands of a binade, and the steps scale with v over the normal range
+// (where the fp16 scale can be nonzero); an infinite v gives NaN, which the
+// caller saturates like infinity.
+__device__ __forceinline__ float div_const(float v, float c, float rc)
+{
+    const float q0 = __fmul_rn(v, rc);
+    const float r = __fmaf_rn(-q0, c, v);
+    return __fmaf_rn(r, rc, q0);
+}
+
 // Scale, zero-point and fast-path parameters of a group from the extremes mn
-// <= 0 <= mx (asymmetric) or the largest magnitude a (symmetric) of its w'.
+// <= 0 <= mx (asymmetric) or the largest magnitude a (symmetric) of its w'
+// (rint(-mn / s16) from quot, like the codes).
 template <int MODE>
 __device__ __forceinline__ QParams group_params(float a, float mn, float mx, unsigned short &s16, bool &exact_only)
 {
     QParams q;
     float s32, hi = 0.f;
-    if (MODE == W4_SYM) s32 = __fdiv_rn(a, 7.0f);
-    else s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-    s16 = (s32 > 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
+    if (MODE == W4_SYM) s32 = div_const(a, 7.0f, __uint_as_float(0x3E124925u));
+    else s32 = div_const(__fsub_rn(mx, mn), 15.0f, __uint_as_float(0x3D888889u));
+    s16 = !(s32 <= 65504.0f) ? (unsigned short)0x7BFF : __half_as_ushort(__float2half_rn(s32));
     q.d = __half2float(__ushort_as_half(s16));
+    q.inv = (q.d > 0.f) ? rcp_approx(q.d) : 0.f;
     if (MODE == W4_SYM) {
         q.zp = 8;
     } else {
-        q.zp = (q.d > 0.f) ? (int)fminf(fmaxf(rintf(__fdiv_rn(-mn, q.d)), 0.f), 15.f) : 0;
+        q.zp = (q.d > 0.f) ? (int)fminf(fmaxf(rintf(quot(-mn, q.inv, q.d)), 0.f), 15.f) : 0;
         hi = (float)(15 - q.zp);
     }
     // the fast path assumes a normal, unsaturated fp16 scale (or a zero one)
     exact_only = (s16 == 0x7BFF) || (q.d > 0.f && q.d < 6.103515625e-05f);
-    q.inv = (q.d > 0.f) ? rcp_approx(q.d) : 0.f;
     q.magic = kMagic + (float)q.zp;              // exact: 1.5*2^23 + zp < 2^24
-    q.hd = (q.d > 0.f) ? 0.5f * q.d : __int_as_float(0x7F800000);
     q.ymax = q.magic + hi;
     return q;
+}
+
+// The fast path's y (magic + code, before any clamp) of one weight.
+template <int MODE>
+__device__ __forceinline__ float fast_y(float x, const QParams &q)
+{
+    const float t = quot(x, q.inv, q.d);
+    if (MODE == W4_SYM) return __fadd_rn(t, q.magic);
+    return __fadd_rn(__fadd_rn(t, kMagic), (float)q.zp);
 }
 
 constexpr int kQItemBytes = 32 * 128;              // one item: 32 slices of 64 bf16
@@ -428,7 +455,13 @@ quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__
         for (int gi = 0; gi < GPL; ++gi) {
             constexpr int WPG = 32 / GPL;        // raw words of the group held by this lane
             float lmin, lmax;                    // extremes of this lane's part of the group (w')
-            if (!FOLD) {                         // on the raw bf16 pairs: one min and one max per pair
+            if (!FOLD && MODE == W4_SYM) {       // on the raw bf16 pairs: one max of magnitudes per pair
+                uint32_t pm = cur[WPG * gi];
+#pragma unroll
+                for (int i = 1; i < WPG; ++i) pm = bmaxabs2(pm, cur[WPG * gi + i]);
+                lmin = 0.f;
+                lmax = fmaxf(fabsf(bf16lo_to_f32(pm)), fabsf(bf16hi_to_f32(pm)));
+            } else if (!FOLD) {                  // one min and one max per pair
                 uint32_t pmin = cur[WPG * gi], pmax = cur[WPG * gi];
 #pragma unroll
                 for (int i = 1; i < WPG; ++i) {
@@ -437,6 +470,13 @@ quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__
                 }
                 lmin = fminf(bf16lo_to_f32(pmin), bf16hi_to_f32(pmin));
                 lmax = fmaxf(bf16lo_to_f32(pmax), bf16hi_to_f32(pmax));
+            } else if (MODE == W4_SYM) {         // folded: the largest magnitude
+                lmin = lmax = 0.f;
+#pragma unroll
+                for (int i = 0; i < WPG; ++i) {
+                    const float2 x = xf[(WPG * gi + i) % (FOLD ? 32 : 1)];
+                    lmax = fmaxf(lmax, fmaxf(fabsf(x.x), fabsf(x.y)));
+                }
             } else {
                 lmin = lmax = 0.f;
 #pragma unroll
@@ -461,55 +501,21 @@ quant_pack_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint32_t *__
             bool eo;
             qp[gi] = group_params<MODE>(a, mn, mx, s16[gi], eo);
             exact_only |= eo;
-            // y is monotonic in w', so when the group's extremes map into [0, 15]
-            // every weight of the group does and no clamp is needed; symmetric
-            // codes never leave [1, 15]: |w'/s16| <= 7 (1 + 2^-11)
+            // rint(w'/s16) is monotonic in w', so when the group's extremes map
+            // into [0, 15] every weight of the group does and no clamp is needed;
+            // symmetric codes never leave [1, 15]: |w'/s16| <= 7 (1 + 2^-11)
             if (MODE == W4_ASYM)
-                clamp |= __fmaf_rn(mn, qp[gi].inv, qp[gi].magic) < kMagic ||
-                         __fmaf_rn(mx, qp[gi].inv, qp[gi].magic) > qp[gi].ymax;
+                clamp |= fast_y<MODE>(mn, qp[gi]) < kMagic || fast_y<MODE>(mx, qp[gi]) > qp[gi].ymax;
         }
 
         // ---- codes ----
-        uint32_t wa[4], wb[4], flags;
-        if (MODE == W4_ASYM && __any_sync(0xffffffffu, clamp))
-            flags = encode<MODE, FOLD, true>(cur, xf, qp[0], wa) |
-                    (encode<MODE, FOLD, true>(cur + 16, xf + (FOLD ? 16 : 0), qp[GPL - 1], wb) << 4);
-        else
-            flags = encode<MODE, FOLD, false>(cur, xf, qp[0], wa) |
-                    (encode<MODE, FOLD, false>(cur + 16, xf + (FOLD ? 16 : 0), qp[GPL - 1], wb) << 4);
-        if (__any_sync(0xffffffffu, flags != 0u)) {
-            // fix the flagged words from the raw weights (read again, from cache)
-            uint32_t m = flags;
-            while (m) {
-                const int w = __ffs(m) - 1;
-                m &= m - 1u;
-                const int c = w >> 2;            // chunk of the word
-                if (c == 1 && !valid1) continue;   // (a half slice's missing chunk is not stored)
-                QParams q = qp[0];
-                if (GPL == 2 && c == 1) q = qp[GPL - 1];
-                const uint4 raw = __ldg((const uint4 *)(src + 4 * w));
-                const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
-                uint32_t word = 0u;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 sp = make_float2(1.f, 1.f);
-                    if (FOLD) {
-                        const float2 *s2 = (const float2 *)(s + 64 * (size_t)cpl) + 4 * w + e;
-                        sp = __ldg(s2);
-                    }
-                    const float2 x = weight_pair<FOLD>(rw[e], sp);
-                    word |= exact_code<MODE>(x.x, q) << nibble_shift(2 * e);
-                    word |= exact_code<MODE>(x.y, q) << nibble_shift(2 * e + 1);
-                }
-                wa[0] = (w == 0) ? word : wa[0];
-                wa[1] = (w == 1) ? word : wa[1];
-                wa[2] = (w == 2) ? word : wa[2];
-                wa[3] = (w == 3) ? word : wa[3];
-                wb[0] = (w == 4) ? word : wb[0];
-                wb[1] = (w == 5) ? word : wb[1];
-                wb[2] = (w == 6) ? word : wb[2];
-                wb[3] = (w == 7) ? word : wb[3];
-            }
+        uint32_t wa[4], wb[4];
+        if (MODE == W4_ASYM && __any_sync(0xffffffffu, clamp)) {
+            encode<MODE, FOLD, true>(cur, xf, qp[0], wa);
+            encode<MODE, FOLD, true>(cur + 16, xf + (FOLD ? 16 : 0), qp[GPL - 1], wb);
+        } else {
+            encode<MODE, FOLD, false>(cur, xf, qp[0], wa);
+            encode<MODE, FOLD, false>(cur + 16, xf + (FOLD ? 16 : 0), qp[GPL - 1], wb);
         }
         if (exact_only) {                        // saturated or subnormal scale: IEEE division
 #pragma unroll
