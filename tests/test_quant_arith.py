@@ -1,4 +1,4 @@
-"""The two arithmetic identities the quantizer's fast path rests on, checked
+"""The arithmetic identities the quantizers' fast paths rest on, checked
 on the CPU by exact emulation of the fp32 steps (numpy float64 holds every
 product and residual exactly; the one sum that does not fit is resolved with
 an error-free TwoSum).
@@ -16,6 +16,10 @@ an error-free TwoSum).
    fp32 x (folded weights, 24 significant bits) on the hardest cases: the 13
    floats nearest h * d for every half-integer h below 32.  Negative x mirror
    positive x (every step is odd in x).
+
+3. The same quotient against the E2M1 rounding midpoints, for bf16 weights
+   and E4M3 block scales (NVFP4): the identity an NVFP4 encoder without a
+   division per weight would rest on.
 
 Each check also runs on a planted mistake (no correction step) and must fail
 there, so that it can fail at all.
@@ -152,3 +156,31 @@ def test_corrected_quotient_on_fp32_weights_next_to_every_half_integer():
         assert np.array_equal(got, want), "inv off by %d ulp" % k
         bad = np.rint(_quot(X, DD, inv, corrected=False).astype(np.float64))
         assert not np.array_equal(bad, want)
+
+
+def test_corrected_quotient_against_the_e2m1_midpoints():
+    """The same corrected quotient for block-scaled FP4 (NVFP4: bf16 weight x,
+    E4M3 block scale s with 4 significant bits): t1 lies on the exact
+    quotient's side of every E2M1 rounding midpoint (0.25 ... 5) and equals
+    the midpoint exactly when x / s does -- for every bf16 x with x / s < 8 and
+    every E4M3 significand (the identity scales with powers of two, E4M3
+    subnormals included), at every reciprocal error from -2 to +2 ulp."""
+    s8 = (1.0 + np.arange(8) / 8.0).astype(np.float32)         # the 8 E4M3 significands of [1, 2)
+    x = _bf16_values(1.0 / 64, 16.0)
+    X, S = np.meshgrid(x, s8, indexing="ij")
+    X, S = X.ravel(), S.ravel()
+    keep = X.astype(np.float64) / S.astype(np.float64) < 8
+    X, S = X[keep], S[keep]
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    # sign(q - m) exactly: x - m * s is exact in float64
+    want = np.sign(X.astype(np.float64)[:, None] - mids[None, :] * S.astype(np.float64)[:, None])
+    assert (want == 0).any()                                  # exact midpoints occur
+    rn = (np.float32(1.0) / S).astype(np.float32)
+    for k in (-2, -1, 0, 1, 2):
+        inv = rn.copy()
+        for _ in range(abs(k)):
+            inv = np.nextafter(inv, np.float32(np.inf if k > 0 else -np.inf)).astype(np.float32)
+        t1 = _quot(X, S, inv).astype(np.float64)
+        assert np.array_equal(np.sign(t1[:, None] - mids[None, :]), want), "inv off by %d ulp" % k
+    t0 = _quot(X, S, rn, corrected=False).astype(np.float64)  # a planted mistake fails
+    assert not np.array_equal(np.sign(t0[:, None] - mids[None, :]), want)
