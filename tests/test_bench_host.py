@@ -62,7 +62,7 @@ def test_max_over_ranks_gloo():
         assert ms == 15.0 and units == 300.0
 
 
-@pytest.mark.parametrize("workload", ["decode", "decodequant", "awq", "fp4quant"])
+@pytest.mark.parametrize("workload", ["decode", "decodequant", "awq", "fp4quant", "mxdecode", "smallbatch"])
 def test_reference_arm_prints_one_complete_line(workload):
     """`bench.py --impl reference` (the CPU oracle on a bounded sample) prints
     one JSON line with the base contract's keys and the same workload
@@ -87,6 +87,26 @@ def test_reference_arm_prints_one_complete_line(workload):
             bench.awq_desc(bench.AWQ_SHAPE["M"], bench.AWQ_SHAPE["N"], bench.AWQ_SHAPE["K"],
                            bench.AWQ_SHAPE["group"], bench.AWQ_SHAPE["n_alpha"]))
     assert d["config"]["workload"] == want
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun with N > 1 the reference arm runs on rank 0 alone: the
+    other ranks exit 0 without work or output, and rank 0's line counts N."""
+    import json
+    import subprocess
+    import sys
+    script = os.path.join(os.path.dirname(bench.__file__), "bench.py")
+    cmd = [sys.executable, script, "--impl", "reference", "--workload", "decode", "--gpus", "2", "--steps", "1",
+           "--warmup", "3"]
+    for rank in (1, 0):
+        env = dict(os.environ, RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE="2")
+        out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env)
+        assert out.returncode == 0, out.stderr[-2000:]
+        lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+        if rank:
+            assert out.stdout.strip() == ""
+        else:
+            assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
 
 
 @pytest.mark.parametrize("workload", ["decode", "decodequant"])
