@@ -55,6 +55,35 @@ int main(void)
     CHECK(w4_awq_search(fake, fake, 16, 256, 8, 128, W4_SYM, 1, (double *)fake, (int *)fake, (float *)fake, fake,
                         1u << 20, stream) == W4_ERR_INVALID_ARG);
 
+    /* the offline repack: sizes by host arithmetic, K % 256 != 0 unsupported */
+    CHECK(w4_repacked_words(16, 256) == 16 * 32);
+    CHECK(w4_repacked_words(17, 256) == 32 * 32);                 /* N padded to whole 16-channel tiles */
+    CHECK(w4_repacked_words(16, 320) == 0);
+    CHECK(w4_repack(NULL, 16, 256, fake_u32, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_repack(fake_u32, 16, 320, fake_u32, stream) == W4_ERR_UNSUPPORTED);
+
+    /* GPTQ: workspace query, then a group size the quantizer does not take */
+    CHECK(w4_gptq_workspace_bytes(64, 256, 128) > 0);
+    CHECK(w4_gptq_workspace_bytes(64, 320, 128) == 0);            /* K not a multiple of the group */
+    CHECK(w4_gptq(fake, fake, 16, 256, 8, 96, W4_SYM, fake_u32, fake, NULL, fake, 1u << 20, stream) ==
+          W4_ERR_INVALID_ARG);
+
+    /* the bf16 rounding of fp32 partial sums */
+    CHECK(w4_f32_to_bf16(NULL, 4, fake, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_f32_to_bf16((const float *)fake, 0, fake, stream) == W4_ERR_INVALID_ARG);
+
+    /* the MX path: block sizes, the tensor-core scale layout's K % 128, flags */
+    CHECK(w4_mxfp8_quant(fake, 1, 48, fake_u8, fake_u8, W4_MX_SCALES_ROWS, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_mxfp8_quant(fake, 1, 96, fake_u8, fake_u8, W4_MX_SCALES_MMA, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_mxfp8_quant(fake, 1, 128, fake_u8, fake_u8, 5, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_mx_scale_layout(fake_u8, 1, 96, fake_u8, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_mx_gemm(fake_u8, fake_u8, 1, 16, 96, fake_u8, fake_u8, fake, 0, stream) == W4_ERR_INVALID_ARG);
+    CHECK(w4_mx_gemm(fake_u8, fake_u8, 1, 16, 128, fake_u8, fake_u8, fake, 3, stream) == W4_ERR_INVALID_ARG);
+
+    /* the failure-path test controls are host settings */
+    w4_set_wait_limit_ns(0);
+    w4_test_stall_first_wait(0);
+
     if (failures == 0) printf("c consumer: all checks held\n");
     return failures == 0 ? 0 : 1;
 }
